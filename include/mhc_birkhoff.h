@@ -1,0 +1,211 @@
+/*
+ * mhc_birkhoff.h -- C ABI of the B200 (sm_100a) kernels for the hot path of
+ * manifold-constrained hyper-connections (mHC): the per-token projection of
+ * 4x4 residual-mixing logits onto the Birkhoff polytope (doubly stochastic
+ * matrices), its implicit backward, and the 4-stream residual mix.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [BA] gist.science summary of arXiv 2606.07574, "Accelerating Birkhoff
+ *        projection for manifold-constrained hyper-connections", §1-§4.
+ *   [DS] deepsignal-app.com, "DeepSeek mHC" article, sections on the Birkhoff
+ *        polytope constraint and the Sinkhorn-Knopp implementation.
+ *   [NA] news.neo-ai.one article 1514, section on doubly stochastic matrices.
+ *   [FP] forpes.ru post 231717, sections "HC" and "mHC".
+ *   [KS] kimiseek.app news on the DeepSeek-V4-Flash analysis, "main changes"
+ *        (mixing maps generated per token from the input).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    allocates nothing, frees nothing and keeps no state between calls apart
+ *    from a per-device cache of the SM count.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL means the legacy default stream) and returns as soon as the work is
+ *    enqueued.
+ *  - Layouts are row-major and contiguous.  A 4x4 matrix is 16 floats (64 B);
+ *    a batch of matrices is [n_mats][4][4].  Residual streams are
+ *    [T][4][C] bfloat16 (given as raw 16-bit patterns, uint16_t), layer
+ *    outputs [T][C] bfloat16, per-token maps [T][4][4] and [T][4] float.
+ *  - Row i of a mixing matrix H is output stream i:  Y_i = sum_j H_ij X_j.
+ *    A row sum of one means each output stream receives one unit in total,
+ *    a column sum of one that each input stream hands out one unit in total
+ *    ([FP] "mHC").
+ *  - Every pointer must be 16-byte aligned (MHC_ERR_ALIGN otherwise); C must
+ *    be a positive multiple of 8 (MHC_ERR_SIZE otherwise).  n_mats == 0 or
+ *    T == 0 returns MHC_OK without launching anything.  Negative sizes return
+ *    MHC_ERR_SIZE.
+ *  - Arguments are validated on the host before any launch; a rejected call
+ *    enqueues nothing.  A failed launch returns MHC_ERR_CUDA.  Faults during
+ *    execution surface at the caller's next synchronisation, as for any CUDA
+ *    kernel.  No kernel traps or asserts.
+ *  - Non-finite logits give NaN in that matrix (and, for the mix, in that
+ *    token's outputs) only.
+ *  - Newton not reaching its tolerance within `iters` iterations is not an
+ *    error: the last iterate is returned (mhc_birkhoff_fwd_diag reports the
+ *    per-matrix iteration counts).
+ *  - Aliasing: P may equal logits, and dlogits may equal dP (each matrix is
+ *    read in full before it is written).  Any other overlap between an input
+ *    and an output is undefined.
+ */
+#ifndef MHC_BIRKHOFF_H
+#define MHC_BIRKHOFF_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+enum mhc_status {
+    MHC_OK = 0,
+    MHC_ERR_NULL = 1,  /* a required pointer is NULL                         */
+    MHC_ERR_ALIGN = 2, /* a pointer is not 16-byte aligned                   */
+    MHC_ERR_SIZE = 3,  /* negative size, C <= 0 or C % 8 != 0, or too large  */
+    MHC_ERR_ARG = 4,   /* unknown method or iteration count out of range     */
+    MHC_ERR_CUDA = 5   /* the CUDA runtime reported an error at launch       */
+};
+
+/* Forward solvers. */
+enum mhc_method {
+    MHC_SINKHORN = 0, /* fixed-count Sinkhorn-Knopp                          */
+    MHC_NEWTON = 1    /* Newton's method on the 3-variable reduced dual      */
+};
+
+/* Largest accepted iteration count for either solver. */
+#define MHC_MAX_ITERS 1000
+
+/*
+ * mhc_birkhoff_fwd -- project each 4x4 logit matrix onto the Birkhoff
+ * polytope.
+ *
+ *   logits  [n_mats][4][4] float, device, read.
+ *   P       [n_mats][4][4] float, device, written.  May alias logits.
+ *   n_mats  number of matrices (>= 0).
+ *   method  MHC_SINKHORN: K = exp(A - rowmax A), then `iters` times divide
+ *             every row by its sum, then every column by its sum
+ *             ([DS] Sinkhorn-Knopp section; [FP] "mHC"; [BA] §1 gives 20 as
+ *             the usual fixed count; [BA] §2.1 the row max shift).  iters = 0
+ *             selects 20.  The result is the algorithm's iterate after
+ *             exactly `iters` rounds, whose row sums need not be 1.
+ *           MHC_NEWTON: the exact projection -- the unique matrix
+ *             P_ij = exp(A_ij + f_i + g_j) with unit row and column sums,
+ *             i.e. the entropic optimal-transport plan with unit marginals
+ *             ([BA] §2) -- found by Newton's method on the dual reduced to the
+ *             three column potentials g_0..g_2 (g_3 = 0) with closed-form
+ *             gradient (column sums minus one) and Hessian ([BA] §2.1).
+ *             `iters` is the maximum Newton iteration count; 0 selects 30.
+ *             Tolerance: every column sum within 1e-6 of one (rows are exact
+ *             to rounding by construction).
+ *   iters   0 .. MHC_MAX_ITERS.
+ *   stream  cudaStream_t or NULL.
+ */
+int mhc_birkhoff_fwd(const float *logits, float *P, int64_t n_mats, int method, int iters,
+                     void *stream);
+
+/*
+ * mhc_birkhoff_fwd_diag -- MHC_NEWTON forward that also writes, per matrix,
+ * the number of Newton iterations taken (a diagnostic for tests and for the
+ * roofline's executed-work count).
+ *
+ *   iters_out [n_mats] int32, device, written.  Other arguments as
+ *   mhc_birkhoff_fwd with method = MHC_NEWTON.
+ */
+int mhc_birkhoff_fwd_diag(const float *logits, float *P, int32_t *iters_out, int64_t n_mats,
+                          int iters, void *stream);
+
+/*
+ * mhc_birkhoff_bwd -- implicit backward of the Newton projection: given the
+ * upstream gradient dP = dL/dP, write dlogits = dL/dlogits.
+ *
+ * By the implicit function theorem ([BA] §2.2), with J the row-softmax
+ * Jacobian at P, S = J[dP] and lambda = H^{-1} colsum(S)[0..2] (lambda_3 = 0),
+ * dlogits = J[dP - 1 lambda^T], where H is the Hessian of the reduced dual at
+ * the solution -- the Hessian of the final Newton iterate ([BA] §2.2,
+ * "Hessian reuse").  H depends on P only, so it is rebuilt from P here; no
+ * iterate of the forward is stored or needed.
+ *
+ *   logits   [n_mats][4][4] float, device, read; used only when P is NULL,
+ *            in which case P is recomputed by the Newton forward in-kernel.
+ *   P        [n_mats][4][4] float, device, read: the forward's output.  May be
+ *            NULL if logits is given.
+ *   dP       [n_mats][4][4] float, device, read.
+ *   dlogits  [n_mats][4][4] float, device, written.  May alias dP.
+ *   At least one of logits and P must be non-NULL (MHC_ERR_NULL otherwise).
+ */
+int mhc_birkhoff_bwd(const float *logits, const float *P, const float *dP, float *dlogits,
+                     int64_t n_mats, void *stream);
+
+/*
+ * mhc_residual_mix_fwd -- Y = H_res . X + h_post (x) F per token:
+ *     Y[t,i,c] = sum_j H_res[t,i,j] X[t,j,c] + h_post[t,i] F[t,c]
+ * The widened residual of n = 4 parallel streams is mixed by the per-token
+ * matrix H_res and the layer output F is written back through the post map
+ * ([FP] "HC" and "mHC"; [KS] per-token maps).  bf16 in and out, fp32
+ * arithmetic, round-to-nearest-even on output.
+ *
+ *   X      [T][4][C] bf16, read.        H_res  [T][4][4] float, read.
+ *   h_post [T][4] float, read.          F      [T][C] bf16, read.
+ *   Y      [T][4][C] bf16, written (must not overlap X or F).
+ *   T >= 0 tokens; C > 0, C % 8 == 0.
+ */
+int mhc_residual_mix_fwd(const uint16_t *X, const float *H_res, const float *h_post,
+                         const uint16_t *F, uint16_t *Y, int64_t T, int64_t C, void *stream);
+
+/*
+ * mhc_residual_mix_bwd -- backward of mhc_residual_mix_fwd for upstream dY:
+ *     dX[t,j,c]   = sum_i H_res[t,i,j] dY[t,i,c]
+ *     dF[t,c]     = sum_i h_post[t,i] dY[t,i,c]
+ *     dH[t,i,j]   = sum_c dY[t,i,c] X[t,j,c]
+ *     dh_post[t,i]= sum_c dY[t,i,c] F[t,c]
+ * and optionally, chained through the projection (H_res must then be the
+ * Newton projection of the logits), dlogits = mhc_birkhoff_bwd(P = H_res,
+ * dP = dH) computed in the same kernel.
+ *
+ *   X, H_res, h_post, F as in the forward; dY [T][4][C] bf16, read.
+ *   dX [T][4][C] bf16, written.  dF [T][C] bf16, written.
+ *   dH_res [T][4][4] float, written, or NULL to skip.
+ *   dh_post [T][4] float, written, or NULL to skip.
+ *   dlogits [T][4][4] float, written, or NULL to skip.
+ *   Reductions over C are accumulated in fp32.
+ */
+int mhc_residual_mix_bwd(const uint16_t *X, const float *H_res, const float *h_post,
+                         const uint16_t *F, const uint16_t *dY, uint16_t *dX, float *dH_res,
+                         float *dh_post, uint16_t *dF, float *dlogits, int64_t T, int64_t C,
+                         void *stream);
+
+/*
+ * mhc_proj_mix_fwd -- fused projection + mix: H_res = Newton projection of
+ * logits (written out for the backward), then Y = H_res . X + h_post (x) F,
+ * in one kernel.  `iters` as for MHC_NEWTON (0 selects 30).
+ *
+ *   logits [T][4][4] float, read.    H_res [T][4][4] float, written.
+ *   Other arguments as mhc_residual_mix_fwd.
+ */
+int mhc_proj_mix_fwd(const float *logits, const float *h_post, const uint16_t *X,
+                     const uint16_t *F, uint16_t *Y, float *H_res, int64_t T, int64_t C,
+                     int iters, void *stream);
+
+/*
+ * mhc_proj_mix_bwd -- fused backward: the mix backward followed, in the same
+ * kernel, by the implicit backward through the projection.
+ *
+ *   H_res [T][4][4] float, read: the projection saved by the forward.
+ *   dlogits [T][4][4] float, written.  dh_post [T][4] float, written.
+ *   dX, dF as in mhc_residual_mix_bwd.
+ */
+int mhc_proj_mix_bwd(const float *H_res, const float *h_post, const uint16_t *X,
+                     const uint16_t *F, const uint16_t *dY, uint16_t *dX, float *dlogits,
+                     float *dh_post, uint16_t *dF, int64_t T, int64_t C, void *stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *mhc_status_string(int status);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int mhc_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MHC_BIRKHOFF_H */
