@@ -1,0 +1,518 @@
+#!/usr/bin/env python
+"""Benchmark of the mHC Birkhoff projection (and, as extras, the residual mix).
+
+Default workload: 131072 fp32 4x4 logit matrices per GPU -- the first half
+N(0,1), the second half N(0,10^2) -- with an N(0,1) upstream gradient.  One
+step is the method's hot path on that batch: the Newton forward (exact
+projection) followed by the implicit backward.  ``value`` is matrices/s for
+that fwd+bwd step, summed over all ranks (weak scaling: every rank owns its own
+shard of matrices; the projection is independent per matrix, so no collective
+runs on the data path).
+
+Timing: W untimed warm-up steps; then, between a barrier and a device
+synchronisation on both sides, exactly K steps, each bracketed by CUDA events
+recorded on the stream the kernels run on, with the L2 cache flushed (a 512 MiB
+write) before every step and outside its events, because the step's 32 MiB
+working set would otherwise stay in the 126 MB L2.  The reported time is the
+sum of the K step durations, maximised over ranks.
+
+Also reported: the end-to-end figure through the public API with host buffers
+(pinned host -> device copies of the inputs and device -> host copies of the
+outputs inside the timed region), the roofline of the dominant kernel against
+the measured HBM copy bandwidth, the fp64 CPU oracle timed on the host cores,
+SM clocks sampled through NVML during the timed region, and (unless
+--no-extras) the 1M/4M/16M sweep, 20-iteration Sinkhorn, and the residual-mix
+workloads.
+
+``--impl reference`` times the fp64 CPU oracle (the reference implementation
+of what the kernels compute) on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "4x4 projections/s (fwd, fwd+bwd) at 128K-16M; mix GB/s vs HBM peak"
+UNIT = "matrices/s"
+WORKLOAD = "birkhoff_fwd_bwd_131072"
+N_MATS = 131072
+BYTES_FWD = 128   # logits in, P out
+BYTES_BWD = 192   # P and dP in, dlogits out
+L2_FLUSH_BYTES = 512 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--no-extras", action="store_true", help="skip the sweep and mix extras")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-oracle sample budget")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- helpers
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def csrc_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "doubly_stochastic_projection_b200", "csrc")
+    for name in sorted(os.listdir(d)):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel
+    sources have not changed since it was captured; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("csrc_hash") != csrc_hash():
+        return None
+    k = d.get("kernels", {}).get(kernel)
+    return None if k is None else k.get("dram_bytes_per_launch_full_size")
+
+
+class ClockSampler:
+    """Polls SM clock and throttle reasons through NVML in a background thread."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index, period=0.01):
+        self.samples = []
+        self.period = period
+        self._stop = threading.Event()
+        self._on = threading.Event()
+        self.max_mhz = None
+        self.ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML unavailable: clocks are reported as unknown
+            self.err = repr(e)
+        self.t = threading.Thread(target=self._run, daemon=True)
+        if self.ok:
+            self.t.start()
+
+    def _run(self):
+        while not self._stop.is_set():
+            if self._on.is_set():
+                try:
+                    mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                    rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.samples.append((mhz, rs))
+                except Exception:
+                    pass
+            time.sleep(self.period)
+
+    def start(self):
+        self._on.set()
+
+    def pause(self):
+        self._on.clear()
+
+    def stop(self):
+        self._stop.set()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": "unavailable"}
+        s = list(self.samples)
+        mhz = [m for m, _ in s]
+        mask = 0
+        for _, r in s:
+            mask |= r
+        reasons = [n for b, n in self.REASONS.items() if mask & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(s), "source": "nvml"}
+
+
+# ----------------------------------------------------------------- distributed
+
+
+def dist_setup(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    return world, rank, local, pg
+
+
+def max_over_ranks(x, pg, device):
+    if pg is None:
+        return x
+    import torch
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg, device):
+    if pg is None:
+        return
+    import torch
+
+    t = torch.zeros(1, device=device)
+    pg.all_reduce(t)
+
+
+# ----------------------------------------------------------------- CPU oracle
+
+
+def cpu_oracle_rate(seconds, n_sample=16384):
+    """fp64 oracle Newton forward + implicit backward on a bounded sample of the
+    workload (matrices of both halves), repeated for about `seconds`."""
+    import numpy as np
+
+    import oracle
+    from doubly_stochastic_projection_b200 import inputs
+
+    A, G = inputs.birkhoff_workload(WORKLOAD)
+    half = n_sample // 2
+    idx = np.concatenate([np.arange(half), N_MATS // 2 + np.arange(half)])
+    A = A[idx].astype(np.float64)
+    G = G[idx].astype(np.float64)
+    oracle.newton(A[:64])
+    done, t0 = 0, time.perf_counter()
+    while True:
+        P = oracle.newton(A, tol=1e-10, max_iter=200)
+        oracle.implicit_bwd(P, G)
+        done += len(A)
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": done / el, "unit": UNIT, "cores": oracle.get_threads(), "kind": "oracle",
+            "sample": "%d matrices (%d of each half of the workload), Newton fwd to ||grad||<1e-10 + "
+                      "implicit bwd in fp64, repeated for %.1f s" % (len(A), half, el)}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+
+    import oracle
+    from doubly_stochastic_projection_b200 import inputs
+
+    A, G = inputs.birkhoff_workload(WORKLOAD)
+    A = A.astype(np.float64)
+    G = G.astype(np.float64)
+    # each step: a bounded sample of the workload, sized so that W + K steps
+    # take about a minute at most
+    total_budget = 60.0
+    per_step = max(64, min(N_MATS, int(2.0e6 * total_budget / max(1, args.steps + args.warmup))))
+    rng = np.random.default_rng(0)
+
+    def step(i):
+        s = (i * per_step) % (N_MATS - per_step + 1)
+        P = oracle.newton(A[s:s + per_step], tol=1e-10, max_iter=200)
+        oracle.implicit_bwd(P, G[s:s + per_step])
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    el = time.perf_counter() - t0
+    value = per_step * args.steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "n_mats": N_MATS, "matrices_per_step_sample": per_step,
+                   "path": "Newton fwd + implicit bwd", "l2": "host"},
+        "cpu_baseline": {"kind": "oracle", "cores": oracle.get_threads(), "value": value, "unit": UNIT,
+                         "sample": "%d consecutive matrices of the workload per step, fp64 Newton fwd + "
+                                   "implicit bwd" % per_step},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- GPU arm
+
+
+def event_time(fn, reps, stream, flush=None):
+    """Mean device time (s) of fn() over reps, events on `stream`, flush outside."""
+    import torch
+
+    tot = 0.0
+    for _ in range(reps):
+        if flush is not None:
+            flush()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        e1.synchronize()
+        tot += e0.elapsed_time(e1) * 1e-3
+    return tot / reps
+
+
+def extras(dev, stream, flush, hbm, api, inputs):
+    import numpy as np
+    import torch
+
+    out = {"sweep": [], "sinkhorn20": [], "mix": []}
+    reps = 5
+    for si, n in enumerate(inputs.SWEEP_SIZES):
+        for di, dist in enumerate(inputs.SWEEP_DISTS):
+            A = torch.from_numpy(inputs.birkhoff_logits(n, dist, inputs.sweep_seed(si, di))).to(dev)
+            G = torch.from_numpy(inputs.upstream_grad(n, inputs.sweep_seed(si, di) + 1000)).to(dev)
+            P = torch.empty_like(A)
+            dl = torch.empty_like(A)
+            api.birkhoff_fwd(A, "newton", out=P)
+            _, its = api.birkhoff_fwd_diag(A)
+            tf = event_time(lambda: api.birkhoff_fwd(A, "newton", out=P), reps, stream, flush)
+            tb = event_time(lambda: api.birkhoff_bwd(G, P=P, out=dl), reps, stream, flush)
+            itn = its.float()
+            out["sweep"].append({
+                "n_mats": n, "dist": dist,
+                "fwd_matrices_per_s": n / tf, "bwd_matrices_per_s": n / tb, "fwd_bwd_matrices_per_s": n / (tf + tb),
+                "fwd_gbs": BYTES_FWD * n / tf / 1e9, "bwd_gbs": BYTES_BWD * n / tb / 1e9,
+                "fwd_frac_hbm": BYTES_FWD * n / tf / 1e9 / hbm, "bwd_frac_hbm": BYTES_BWD * n / tb / 1e9 / hbm,
+                "fwd_bwd_frac_hbm": (BYTES_FWD + BYTES_BWD) * n / (tf + tb) / 1e9 / hbm,
+                "newton_iters_mean": float(itn.mean()), "newton_iters_max": int(its.max()),
+                "newton_iters_warp_max_mean": float(itn.reshape(-1, 32).max(1).values.mean()),
+            })
+            if dist in ("normal1", "normal10"):
+                ts = event_time(lambda: api.birkhoff_fwd(A, "sinkhorn", 20, out=P), reps, stream, flush)
+                out["sinkhorn20"].append({"n_mats": n, "dist": dist, "fwd_matrices_per_s": n / ts,
+                                          "fwd_gbs": BYTES_FWD * n / ts / 1e9,
+                                          "fwd_frac_hbm": BYTES_FWD * n / ts / 1e9 / hbm})
+            del A, G, P, dl, its
+            torch.cuda.empty_cache()
+    for name in ("mix_T16384_C4096", "mix_T65536_C7168"):
+        m = inputs.mix_workload(name, device=dev)
+        T, C = m["T"], m["C"]
+        X, F, dY = m["X"], m["F"], m["dY"]
+        lg = torch.from_numpy(m["logits"]).to(dev)
+        h = torch.from_numpy(m["h_post"]).to(dev)
+        Y = torch.empty_like(X)
+        H = api.birkhoff_fwd(lg, "newton")
+        tf = event_time(lambda: api.residual_mix_fwd(X, H, h, F, out=Y), reps, stream, flush)
+        tb = event_time(lambda: api.residual_mix_bwd(X, H, h, F, dY, need_dlogits=True), reps, stream, flush)
+        tff = event_time(lambda: api.proj_mix_fwd(lg, h, X, F, out=Y, H_out=H), reps, stream, flush)
+        tfb = event_time(lambda: api.proj_mix_bwd(H, h, X, F, dY), reps, stream, flush)
+        bf = (18 * C + 80) * T
+        bb = (28 * C + 160) * T
+        bff = (18 * C + 128) * T          # + logits in, H out instead of H in
+        bfb = (28 * C + 160) * T          # dH not written, dlogits written
+        out["mix"].append({
+            "workload": name, "T": T, "C": C,
+            "fwd_gbs": bf / tf / 1e9, "fwd_frac_hbm": bf / tf / 1e9 / hbm, "fwd_tokens_per_s": T / tf,
+            "bwd_gbs": bb / tb / 1e9, "bwd_frac_hbm": bb / tb / 1e9 / hbm, "bwd_tokens_per_s": T / tb,
+            "fused_fwd_gbs": bff / tff / 1e9, "fused_fwd_frac_hbm": bff / tff / 1e9 / hbm,
+            "fused_bwd_gbs": bfb / tfb / 1e9, "fused_bwd_frac_hbm": bfb / tfb / 1e9 / hbm,
+            "fused_fwd_bwd_tokens_per_s": T / (tff + tfb),
+        })
+        del m, X, F, dY, Y, H, lg, h
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_b200(args):
+    import numpy as np
+    import torch
+
+    from doubly_stochastic_projection_b200 import api, inputs
+
+    world, rank, local, pg = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    api.lib()
+    stream = torch.cuda.current_stream(dev)
+    hbm, hbm_src = measured_peaks()
+
+    # this rank's shard: same distributions, its own seeds
+    A_np, G_np = inputs.birkhoff_workload(WORKLOAD)
+    if rank:
+        A_np = inputs.birkhoff_logits(N_MATS, "halves_1_10", 2 + 7919 * rank)
+        G_np = inputs.upstream_grad(N_MATS, 102 + 7919 * rank)
+    A = torch.from_numpy(A_np).to(dev)
+    G = torch.from_numpy(G_np).to(dev)
+    P = torch.empty_like(A)
+    dl = torch.empty_like(A)
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.zero_()
+
+    def step():
+        api.birkhoff_fwd(A, "newton", out=P)
+        api.birkhoff_bwd(G, P=P, out=dl)
+
+    for _ in range(max(3, args.warmup)):
+        flush()
+        step()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(pg, dev)
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(K):
+        flush()
+        e0, e1, e2 = ev[i]
+        e0.record(stream)
+        api.birkhoff_fwd(A, "newton", out=P)
+        e1.record(stream)
+        api.birkhoff_bwd(G, P=P, out=dl)
+        e2.record(stream)
+    torch.cuda.synchronize()
+    clocks.pause()
+    barrier(pg, dev)
+    t_fwd = sum(e0.elapsed_time(e1) for e0, e1, _ in ev) * 1e-3
+    t_bwd = sum(e1.elapsed_time(e2) for _, e1, e2 in ev) * 1e-3
+    t_step = t_fwd + t_bwd
+    t_max = max_over_ranks(t_step, pg, dev)
+    value = world * N_MATS * K / t_max
+    gpu_launches = 2 * K
+
+    # end to end through the public API, host buffers, copies timed
+    A_h = A.cpu().pin_memory()
+    G_h = G.cpu().pin_memory()
+    P_h = torch.empty_like(A_h).pin_memory()
+    dl_h = torch.empty_like(A_h).pin_memory()
+    A_d = torch.empty_like(A)
+    G_d = torch.empty_like(G)
+    e2e_steps = max(3, min(K, 200))
+    for _ in range(3):
+        A_d.copy_(A_h, non_blocking=True)
+    torch.cuda.synchronize()
+    tot = 0.0
+    for i in range(e2e_steps):
+        flush()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        A_d.copy_(A_h, non_blocking=True)
+        G_d.copy_(G_h, non_blocking=True)
+        api.birkhoff_fwd(A_d, "newton", out=P)
+        api.birkhoff_bwd(G_d, P=P, out=dl)
+        P_h.copy_(P, non_blocking=True)
+        dl_h.copy_(dl, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        tot += e0.elapsed_time(e1) * 1e-3
+    t_e2e = max_over_ranks(tot / e2e_steps, pg, dev)
+    e2e = {"value": world * N_MATS / t_e2e, "unit": UNIT, "h2d_bytes_per_step": 2 * A.numel() * 4,
+           "d2h_bytes_per_step": 2 * A.numel() * 4,
+           "path": "pinned host -> device copies, Newton fwd, implicit bwd, device -> host copies of P and dlogits"}
+
+    # dominant kernel and its roofline (HBM-bound: algorithmic bytes / time)
+    if t_fwd >= t_bwd:
+        kname, kbytes, kt = "newton_fwd_kernel", BYTES_FWD * N_MATS, t_fwd / K
+    else:
+        kname, kbytes, kt = "implicit_bwd_kernel", BYTES_BWD * N_MATS, t_bwd / K
+    achieved = kbytes / kt / 1e9
+    traffic = profiled_traffic(kname)
+    roofline = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": traffic, "peak_source": hbm_src,
+                "algorithmic_bytes_per_launch": kbytes, "launch_us": kt * 1e6,
+                "note": "peak is the %s HBM copy bandwidth; the kernel is timed in isolation" % hbm_src}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": 1e3 * t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "n_mats_per_gpu": N_MATS,
+                   "logits": "first half N(0,1), second half N(0,10^2), seed 2 (+7919*rank)",
+                   "step": "Newton fwd (to max|colsum-1|<1e-6) + implicit bwd",
+                   "l2": "flushed (512 MiB write) before every step, outside its events",
+                   "parallelism": "token-sharded replicas, no collective" if world > 1 else "single GPU"},
+        "fwd_matrices_per_s": world * N_MATS * K / max_over_ranks(t_fwd, pg, dev),
+        "bwd_matrices_per_s": world * N_MATS * K / max_over_ranks(t_bwd, pg, dev),
+        "e2e": e2e, "gpu_launches": gpu_launches, "roofline": roofline,
+    }
+
+    line["clocks"] = clocks.summary()
+    if rank == 0 and not args.no_extras:
+        clocks.samples = []
+        clocks.start()
+        try:
+            line["extras"] = extras(dev, stream, flush, hbm, api, inputs)
+            # SK-20 on the default workload, for comparison
+            tsk = event_time(lambda: api.birkhoff_fwd(A, "sinkhorn", 20, out=P), 20, stream, flush)
+            line["extras"]["sinkhorn20_default_workload_matrices_per_s"] = N_MATS / tsk
+        finally:
+            clocks.pause()
+        line["extras"]["clocks"] = clocks.summary()
+    clocks.stop()
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_rate(args.cpu_seconds)
+    elif rank == 0:
+        line["cpu_baseline"] = None
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        barrier(pg, dev)
+        pg.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_b200(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

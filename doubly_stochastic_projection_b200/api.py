@@ -1,0 +1,235 @@
+"""Python binding of ``libmhc_b200.so`` (C ABI in ``include/mhc_birkhoff.h``).
+
+Argument marshalling only: each function checks that its tensors are CUDA,
+contiguous and of the right dtype, allocates outputs with torch (device memory
+is torch's job here), and calls the C entry point of the same name on the
+current CUDA stream.  Every step of the computation runs in the library's
+kernels; there is no CPU or PyTorch fallback, and a missing library raises.
+
+bf16 tensors are handed to the library as raw 16-bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import build as _build
+
+SINKHORN = 0
+NEWTON = 1
+_METHODS = {"sinkhorn": SINKHORN, "newton": NEWTON, SINKHORN: SINKHORN, NEWTON: NEWTON}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class MhcError(RuntimeError):
+    """A non-zero status returned by the C library."""
+
+    def __init__(self, status: int, msg: str):
+        super().__init__(msg)
+        self.status = status
+
+
+def library_path() -> str:
+    return _build.LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library (once).  Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.LIB_PATH
+            if not os.path.exists(path):
+                raise RuntimeError(
+                    "%s is missing: build it with `python -m doubly_stochastic_projection_b200.build` "
+                    "or __graft_entry__.build(); there is no fallback implementation" % path)
+            L = ctypes.CDLL(path)
+            p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+            sig = {
+                "mhc_birkhoff_fwd": [p, p, i64, i32, i32, p],
+                "mhc_birkhoff_fwd_diag": [p, p, p, i64, i32, p],
+                "mhc_birkhoff_bwd": [p, p, p, p, i64, p],
+                "mhc_residual_mix_fwd": [p, p, p, p, p, i64, i64, p],
+                "mhc_residual_mix_bwd": [p, p, p, p, p, p, p, p, p, p, i64, i64, p],
+                "mhc_proj_mix_fwd": [p, p, p, p, p, p, i64, i64, i32, p],
+                "mhc_proj_mix_bwd": [p, p, p, p, p, p, p, p, p, i64, i64, p],
+            }
+            for name, args in sig.items():
+                f = getattr(L, name)
+                f.argtypes = args
+                f.restype = ctypes.c_int
+            L.mhc_status_string.argtypes = [ctypes.c_int]
+            L.mhc_status_string.restype = ctypes.c_char_p
+            L.mhc_version.argtypes = []
+            L.mhc_version.restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().mhc_status_string(int(status)).decode()
+
+
+def _check(rc: int) -> None:
+    if rc != 0:
+        raise MhcError(rc, status_string(rc))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _need(t, name, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor (there is no CPU implementation)" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    return t
+
+
+def _n_mats(logits):
+    if logits.dim() < 2 or tuple(logits.shape[-2:]) != (4, 4):
+        raise ValueError("expected [..., 4, 4] matrices, got %s" % (tuple(logits.shape),))
+    return logits.numel() // 16
+
+
+def birkhoff_fwd(logits: torch.Tensor, method="newton", iters: int = 0, out: torch.Tensor | None = None):
+    """Project [..., 4, 4] float32 logits onto the Birkhoff polytope.
+
+    ``method``: "newton" (exact projection by Newton on the 3-variable reduced
+    dual; ``iters`` = maximum iterations, 0 -> 30) or "sinkhorn" (exactly
+    ``iters`` Sinkhorn-Knopp rounds, 0 -> 20).
+    """
+    _need(logits, "logits", torch.float32)
+    n = _n_mats(logits)
+    if out is None:
+        out = torch.empty_like(logits)
+    _need(out, "out", torch.float32, logits.shape)
+    m = _METHODS.get(method, -1) if not isinstance(method, int) else method
+    _check(lib().mhc_birkhoff_fwd(_ptr(logits), _ptr(out), n, int(m), int(iters), _stream(logits)))
+    return out
+
+
+def birkhoff_fwd_diag(logits: torch.Tensor, iters: int = 0):
+    """Newton forward that also returns the per-matrix iteration counts (int32)."""
+    _need(logits, "logits", torch.float32)
+    n = _n_mats(logits)
+    out = torch.empty_like(logits)
+    its = torch.empty(logits.shape[:-2], dtype=torch.int32, device=logits.device)
+    _check(lib().mhc_birkhoff_fwd_diag(_ptr(logits), _ptr(out), _ptr(its), n, int(iters), _stream(logits)))
+    return out, its
+
+
+def birkhoff_bwd(dP: torch.Tensor, P: torch.Tensor | None = None, logits: torch.Tensor | None = None,
+                 out: torch.Tensor | None = None):
+    """Implicit backward: dlogits from the upstream dP and the saved projection P
+    (or, when P is None, from the logits, recomputing P in-kernel)."""
+    _need(dP, "dP", torch.float32)
+    n = _n_mats(dP)
+    if P is not None:
+        _need(P, "P", torch.float32, dP.shape)
+    if logits is not None:
+        _need(logits, "logits", torch.float32, dP.shape)
+    if out is None:
+        out = torch.empty_like(dP)
+    _need(out, "out", torch.float32, dP.shape)
+    _check(lib().mhc_birkhoff_bwd(_ptr(logits), _ptr(P), _ptr(dP), _ptr(out), n, _stream(dP)))
+    return out
+
+
+def _mix_shapes(X, F):
+    _need(X, "X", torch.bfloat16)
+    if X.dim() != 3 or X.shape[1] != 4:
+        raise ValueError("X must be [T, 4, C], got %s" % (tuple(X.shape),))
+    T, _, C = X.shape
+    _need(F, "F", torch.bfloat16, (T, C))
+    return T, C
+
+
+def residual_mix_fwd(X, H_res, h_post, F, out=None):
+    """Y[t,i,c] = sum_j H_res[t,i,j] X[t,j,c] + h_post[t,i] F[t,c] (bf16 in/out)."""
+    T, C = _mix_shapes(X, F)
+    _need(H_res, "H_res", torch.float32, (T, 4, 4))
+    _need(h_post, "h_post", torch.float32, (T, 4))
+    if out is None:
+        out = torch.empty_like(X)
+    _need(out, "out", torch.bfloat16, X.shape)
+    _check(lib().mhc_residual_mix_fwd(_ptr(X), _ptr(H_res), _ptr(h_post), _ptr(F), _ptr(out), T, C,
+                                      _stream(X)))
+    return out
+
+
+def residual_mix_bwd(X, H_res, h_post, F, dY, need_dH=True, need_dh_post=True, need_dlogits=False):
+    """Backward of the mix.  Returns a dict with dX, dF and, as requested, dH_res,
+    dh_post and dlogits (the latter chained through the implicit projection
+    backward with P = H_res)."""
+    T, C = _mix_shapes(X, F)
+    _need(H_res, "H_res", torch.float32, (T, 4, 4))
+    _need(h_post, "h_post", torch.float32, (T, 4))
+    _need(dY, "dY", torch.bfloat16, X.shape)
+    dX = torch.empty_like(X)
+    dF = torch.empty_like(F)
+    dH = torch.empty_like(H_res) if need_dH else None
+    dh = torch.empty_like(h_post) if need_dh_post else None
+    dl = torch.empty_like(H_res) if need_dlogits else None
+    _check(lib().mhc_residual_mix_bwd(_ptr(X), _ptr(H_res), _ptr(h_post), _ptr(F), _ptr(dY), _ptr(dX),
+                                      _ptr(dH), _ptr(dh), _ptr(dF), _ptr(dl), T, C, _stream(X)))
+    return {"dX": dX, "dF": dF, "dH_res": dH, "dh_post": dh, "dlogits": dl}
+
+
+def proj_mix_fwd(logits, h_post, X, F, iters: int = 0, out=None, H_out=None):
+    """Fused Newton projection + mix.  Returns (Y, H_res)."""
+    T, C = _mix_shapes(X, F)
+    _need(logits, "logits", torch.float32, (T, 4, 4))
+    _need(h_post, "h_post", torch.float32, (T, 4))
+    Y = torch.empty_like(X) if out is None else _need(out, "out", torch.bfloat16, X.shape)
+    H = torch.empty_like(logits) if H_out is None else _need(H_out, "H_out", torch.float32, (T, 4, 4))
+    _check(lib().mhc_proj_mix_fwd(_ptr(logits), _ptr(h_post), _ptr(X), _ptr(F), _ptr(Y), _ptr(H), T, C,
+                                  int(iters), _stream(X)))
+    return Y, H
+
+
+def proj_mix_bwd(H_res, h_post, X, F, dY):
+    """Fused mix backward + implicit projection backward.
+    Returns (dX, dlogits, dh_post, dF)."""
+    T, C = _mix_shapes(X, F)
+    _need(H_res, "H_res", torch.float32, (T, 4, 4))
+    _need(h_post, "h_post", torch.float32, (T, 4))
+    _need(dY, "dY", torch.bfloat16, X.shape)
+    dX = torch.empty_like(X)
+    dF = torch.empty_like(F)
+    dl = torch.empty_like(H_res)
+    dh = torch.empty_like(h_post)
+    _check(lib().mhc_proj_mix_bwd(_ptr(H_res), _ptr(h_post), _ptr(X), _ptr(F), _ptr(dY), _ptr(dX), _ptr(dl),
+                                  _ptr(dh), _ptr(dF), T, C, _stream(X)))
+    return dX, dl, dh, dF
+
+
+class BirkhoffProjection(torch.autograd.Function):
+    """Autograd wrapper: Newton forward, implicit backward (saves P only)."""
+
+    @staticmethod
+    def forward(ctx, logits, iters: int = 0):
+        P = birkhoff_fwd(logits.contiguous(), "newton", iters)
+        ctx.save_for_backward(P)
+        return P
+
+    @staticmethod
+    def backward(ctx, dP):
+        (P,) = ctx.saved_tensors
+        return birkhoff_bwd(dP.contiguous(), P=P), None

@@ -1,0 +1,345 @@
+// birkhoff_math.cuh -- per-matrix device arithmetic of the 4x4 Birkhoff
+// projection: the Sinkhorn-Knopp and Newton forward solvers and the implicit
+// backward.  One thread owns one 4x4 matrix in 16 registers; there is no
+// shared or global memory traffic inside these routines.
+//
+// Sources:
+//   [BA] gist.science summary of arXiv 2606.07574, "Accelerating Birkhoff
+//        projection for manifold-constrained hyper-connections".
+//   [DS] deepsignal-app.com "DeepSeek mHC" article, Sinkhorn-Knopp section.
+//
+// Layout: a[4*r + c] is row r, column c.  Row r of the projected matrix is
+// output stream r of the residual mix.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mhc {
+
+constexpr int kDefaultNewtonIters = 30;
+constexpr int kDefaultSinkhornIters = 20;
+// Newton stops once every column sum is within this of one (rows are
+// normalised exactly, up to rounding, at every iterate).
+constexpr float kNewtonTol = 1e-6f;
+// Armijo backtracking is used while the column-sum error is at least this;
+// below it full Newton steps are taken (quadratic region).
+constexpr float kLineSearchAbove = 1e-2f;
+constexpr float kArmijo = 1e-4f;
+constexpr int kMaxHalvings = 24;
+// No dual potential moves by more than this (in log units) per iteration.
+constexpr float kStepCap = 16.0f;
+
+__device__ __forceinline__ float rcp_rn(float x) { return __frcp_rn(x); }
+
+__device__ __forceinline__ void load16(const float* p, float (&a)[16])
+{
+    const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const float4 v = __ldg(q + r);
+        a[4 * r + 0] = v.x;
+        a[4 * r + 1] = v.y;
+        a[4 * r + 2] = v.z;
+        a[4 * r + 3] = v.w;
+    }
+}
+
+__device__ __forceinline__ void store16(float* p, const float (&a)[16])
+{
+    float4* q = reinterpret_cast<float4*>(p);
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+        q[r] = make_float4(a[4 * r + 0], a[4 * r + 1], a[4 * r + 2], a[4 * r + 3]);
+}
+
+__device__ __forceinline__ void normalize_rows(float (&a)[16])
+{
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const float s = (a[4 * r] + a[4 * r + 1]) + (a[4 * r + 2] + a[4 * r + 3]);
+        const float q = rcp_rn(s);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) a[4 * r + c] *= q;
+    }
+}
+
+__device__ __forceinline__ void normalize_cols(float (&a)[16])
+{
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const float s = (a[c] + a[4 + c]) + (a[8 + c] + a[12 + c]);
+        const float q = rcp_rn(s);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) a[4 * r + c] *= q;
+    }
+}
+
+__device__ __forceinline__ void shift_rows_by_max(float (&a)[16])
+{
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const float m = fmaxf(fmaxf(a[4 * r], a[4 * r + 1]), fmaxf(a[4 * r + 2], a[4 * r + 3]));
+#pragma unroll
+        for (int c = 0; c < 4; ++c) a[4 * r + c] -= m;
+    }
+}
+
+__device__ __forceinline__ void shift_cols_by_max(float (&a)[16])
+{
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const float m = fmaxf(fmaxf(a[c], a[4 + c]), fmaxf(a[8 + c], a[12 + c]));
+#pragma unroll
+        for (int r = 0; r < 4; ++r) a[4 * r + c] -= m;
+    }
+}
+
+__device__ __forceinline__ bool all_finite(const float (&a)[16])
+{
+    bool ok = true;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) ok = ok && isfinite(a[k]);
+    return ok;
+}
+
+__device__ __forceinline__ void fill_nan(float (&a)[16])
+{
+#pragma unroll
+    for (int k = 0; k < 16; ++k) a[k] = __int_as_float(0x7fffffff);
+}
+
+// ---------------------------------------------------------------------------
+// The dual Hessian as a grounded graph Laplacian.
+//
+// With rows of P summing to one, the Hessian of the reduced dual ([BA] §2.1)
+//     H_jk = sum_i P_ij (delta_jk - P_ik),   j, k in {0, 1, 2}
+// equals the Laplacian of the complete graph on the four columns with edge
+// weights w_jk = sum_i P_ij P_ik, with column 3 (whose potential is fixed at
+// zero) as ground: H_jk = -w_jk off the diagonal and H_jj = sum_{k != j} w_jk.
+// Solving H x = r by eliminating nodes 0 and 1 in turn only ever adds positive
+// weights (Kron reduction; the Grassmann-Taksar-Heyman form of Gaussian
+// elimination), so no pivot is formed by cancellation even when P is close to
+// a permutation and every weight is tiny.
+// ---------------------------------------------------------------------------
+struct PairWeights {
+    float w01, w02, w03, w12, w13, w23;
+};
+
+__device__ __forceinline__ PairWeights pair_weights(const float (&p)[16])
+{
+    PairWeights w;
+    w.w01 = p[0] * p[1];
+    w.w02 = p[0] * p[2];
+    w.w03 = p[0] * p[3];
+    w.w12 = p[1] * p[2];
+    w.w13 = p[1] * p[3];
+    w.w23 = p[2] * p[3];
+#pragma unroll
+    for (int r = 1; r < 4; ++r) {
+        const float* q = p + 4 * r;
+        w.w01 = fmaf(q[0], q[1], w.w01);
+        w.w02 = fmaf(q[0], q[2], w.w02);
+        w.w03 = fmaf(q[0], q[3], w.w03);
+        w.w12 = fmaf(q[1], q[2], w.w12);
+        w.w13 = fmaf(q[1], q[3], w.w13);
+        w.w23 = fmaf(q[2], q[3], w.w23);
+    }
+    return w;
+}
+
+// Solves H x = r for the grounded Laplacian above.  Returns false when a pivot
+// is not a positive finite number (an isolated column).
+__device__ __forceinline__ bool laplacian_solve(const PairWeights& w, float r0, float r1, float r2,
+                                                float& x0, float& x1, float& x2)
+{
+    const float a = (w.w01 + w.w02) + w.w03;
+    const float ia = rcp_rn(a);
+    // eliminate node 0: reduced weights among nodes 1, 2 and ground
+    const float v12 = fmaf(w.w01 * w.w02, ia, w.w12);
+    const float v13 = fmaf(w.w01 * w.w03, ia, w.w13);
+    const float v23 = fmaf(w.w02 * w.w03, ia, w.w23);
+    const float q1 = fmaf(w.w01 * r0, ia, r1);
+    const float q2 = fmaf(w.w02 * r0, ia, r2);
+    // eliminate node 1
+    const float b = v12 + v13;
+    const float ib = rcp_rn(b);
+    const float u = fmaf(v12 * v13, ib, v23);
+    const float q2b = fmaf(v12 * q1, ib, q2);
+    x2 = q2b * rcp_rn(u);
+    x1 = fmaf(v12, x2, q1) * ib;
+    x0 = fmaf(w.w01, x1, fmaf(w.w02, x2, r0)) * ia;
+    const bool piv = (a > 0.0f) && (b > 0.0f) && (u > 0.0f) && (ia <= 3.0e38f) &&
+                     (ib <= 3.0e38f);
+    return piv && isfinite(x0) && isfinite(x1) && isfinite(x2);
+}
+
+// ---------------------------------------------------------------------------
+// Forward solver 1: Sinkhorn-Knopp with a fixed iteration count.
+// K = exp(A - rowmax A) ([BA] §2.1 max shift), then `iters` rounds of
+// "divide every row by its sum, then every column by its sum" ([DS]; [BA] §1
+// names 20 as the usual fixed count).  Division is done as multiplication by
+// a correctly rounded reciprocal.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void sinkhorn_project(float (&a)[16], int iters)
+{
+    shift_rows_by_max(a);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) a[k] = expf(a[k]);
+    for (int it = 0; it < iters; ++it) {
+        normalize_rows(a);
+        normalize_cols(a);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Forward solver 2: Newton's method on the 3-variable reduced dual ([BA] §2,
+// §2.1).  The projection is P_ij = exp(A_ij + f_i + g_j) with unit row and
+// column sums.  Eliminating f leaves the convex
+//     phi(g) = sum_i logsumexp_j(A_ij + g_j) - sum_j g_j,   g_3 = 0,
+// whose gradient is colsum(P) - 1 and whose Hessian is the Laplacian above.
+//
+// The iterate is held as P itself (rows normalised), not as g: a step d
+// multiplies column j by exp(t d_j) and renormalises the rows, which is the
+// same map as g += t d but keeps every entry in [0, 1] and needs three exps
+// per step instead of sixteen.  Start: A shifted by its row maxima and then
+// its column maxima (P is unchanged by either, [BA] §2.1 shift redundancy and
+// max shift), exponentiated, rows normalised, then one Sinkhorn round as a
+// warm start.  Globalisation: the step is capped at kStepCap per potential,
+// Armijo backtracking on phi while the error is large; a Sinkhorn round
+// replaces the step when the Laplacian is singular or no decrease is found.
+// Returns the number of Newton iterations taken.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int newton_project(float (&a)[16], int maxit)
+{
+    if (!all_finite(a)) {
+        fill_nan(a);
+        return 0;
+    }
+    shift_rows_by_max(a);
+    shift_cols_by_max(a);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) a[k] = expf(a[k]);
+    normalize_rows(a);
+    normalize_cols(a);
+    normalize_rows(a);
+
+    int it = 0;
+    for (; it < maxit; ++it) {
+        const float c0 = (a[0] + a[4]) + (a[8] + a[12]);
+        const float c1 = (a[1] + a[5]) + (a[9] + a[13]);
+        const float c2 = (a[2] + a[6]) + (a[10] + a[14]);
+        const float c3 = (a[3] + a[7]) + (a[11] + a[15]);
+        const float g0 = c0 - 1.0f, g1 = c1 - 1.0f, g2 = c2 - 1.0f;
+        const float err = fmaxf(fmaxf(fabsf(g0), fabsf(g1)), fmaxf(fabsf(g2), fabsf(c3 - 1.0f)));
+        if (!(err >= kNewtonTol)) break;
+
+        const PairWeights w = pair_weights(a);
+        float d0, d1, d2;
+        bool ok = laplacian_solve(w, -g0, -g1, -g2, d0, d1, d2);
+        const float dmax = fmaxf(fmaxf(fabsf(d0), fabsf(d1)), fabsf(d2));
+        if (ok && dmax > kStepCap) {
+            const float s = kStepCap / dmax;
+            d0 *= s;
+            d1 *= s;
+            d2 *= s;
+        }
+        float e0 = 1.0f, e1 = 1.0f, e2 = 1.0f;
+        if (ok) {
+            e0 = expf(d0);
+            e1 = expf(d1);
+            e2 = expf(d2);
+            if (err >= kLineSearchAbove) {
+                // phi(g + t d) - phi(g) = sum_i log(sum_j P_ij e^{t d_j}) - t sum_j d_j
+                const float slope = fmaf(g0, d0, fmaf(g1, d1, g2 * d2));
+                const float dsum = (d0 + d1) + d2;
+                float t = 1.0f;
+                ok = false;
+                for (int h = 0; h < kMaxHalvings && slope < 0.0f; ++h) {
+                    float prod = 1.0f;
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const float s =
+                            fmaf(a[4 * r], e0, fmaf(a[4 * r + 1], e1, fmaf(a[4 * r + 2], e2, a[4 * r + 3])));
+                        prod *= s;
+                    }
+                    const float dphi = logf(prod) - t * dsum;
+                    if (dphi <= kArmijo * t * slope) {
+                        ok = true;
+                        break;
+                    }
+                    t *= 0.5f;
+                    e0 = expf(t * d0);
+                    e1 = expf(t * d1);
+                    e2 = expf(t * d2);
+                }
+            }
+        }
+        if (ok) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                a[4 * r + 0] *= e0;
+                a[4 * r + 1] *= e1;
+                a[4 * r + 2] *= e2;
+            }
+            normalize_rows(a);
+        } else {
+            normalize_cols(a);
+            normalize_rows(a);
+        }
+    }
+    return it;
+}
+
+// ---------------------------------------------------------------------------
+// Implicit backward ([BA] §2.2).  For upstream G = dL/dP at the projection P:
+//     S = J[G],  lambda = H^{-1} colsum(S)[0..2] (lambda_3 = 0),
+//     dL/dA = J[G - 1 lambda^T],
+// where J is the row-softmax Jacobian at P and H the dual Hessian at the
+// solution -- the Hessian of the last Newton iterate ("Hessian reuse"),
+// rebuilt here from P.  J is applied in pairwise form,
+//     J[X]_ik = P_ik sum_{j != k} P_ij (X_ik - X_ij),
+// which equals P_ik (X_ik - sum_j P_ij X_ij) for unit row sums but never
+// subtracts two nearly equal weighted means: for P close to a permutation
+// the weighted-mean form loses all relative accuracy in fp32.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void implicit_vjp(const float (&p)[16], const float (&g)[16],
+                                             float (&out)[16])
+{
+    float D[4][6];
+    float c0 = 0.0f, c1 = 0.0f, c2 = 0.0f;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const float* x = g + 4 * r;
+        const float* q = p + 4 * r;
+        D[r][0] = x[0] - x[1];
+        D[r][1] = x[0] - x[2];
+        D[r][2] = x[0] - x[3];
+        D[r][3] = x[1] - x[2];
+        D[r][4] = x[1] - x[3];
+        D[r][5] = x[2] - x[3];
+        c0 = fmaf(q[0], fmaf(q[1], D[r][0], fmaf(q[2], D[r][1], q[3] * D[r][2])), c0);
+        c1 = fmaf(q[1], fmaf(q[2], D[r][3], fmaf(q[3], D[r][4], -q[0] * D[r][0])), c1);
+        c2 = fmaf(q[2], fmaf(q[3], D[r][5], fmaf(-q[0], D[r][1], -q[1] * D[r][3])), c2);
+    }
+    float l0, l1, l2;
+    const bool ok = laplacian_solve(pair_weights(p), c0, c1, c2, l0, l1, l2);
+    if (!ok) {
+        fill_nan(out);
+        return;
+    }
+    const float L[6] = {l0 - l1, l0 - l2, l0, l1 - l2, l1, l2};
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const float* q = p + 4 * r;
+        float E[6];
+#pragma unroll
+        for (int k = 0; k < 6; ++k) E[k] = D[r][k] - L[k];
+        out[4 * r + 0] = q[0] * fmaf(q[1], E[0], fmaf(q[2], E[1], q[3] * E[2]));
+        out[4 * r + 1] = q[1] * fmaf(q[2], E[3], fmaf(q[3], E[4], -q[0] * E[0]));
+        out[4 * r + 2] = q[2] * fmaf(q[3], E[5], fmaf(-q[0], E[1], -q[1] * E[3]));
+        out[4 * r + 3] = q[3] * fmaf(-q[0], E[2], fmaf(-q[1], E[4], -q[2] * E[5]));
+    }
+}
+
+}  // namespace mhc

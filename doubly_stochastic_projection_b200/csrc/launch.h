@@ -1,0 +1,33 @@
+// launch.h -- internal launchers behind the C ABI (not installed).  Each
+// returns the CUDA error of its launch; argument validation happens in
+// mhc_api.cu before any of these is called.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mhc {
+
+// Number of SMs of the current device (cached per device).
+int device_sm_count();
+
+// Grid size for a grid-stride kernel: enough CTAs to fill every SM at the
+// kernel's occupancy, never more than `blocks_needed`.
+int persistent_grid(const void* kernel, int threads, size_t smem, int64_t blocks_needed);
+
+cudaError_t launch_sinkhorn_fwd(const float* logits, float* P, int64_t n, int iters, cudaStream_t s);
+cudaError_t launch_newton_fwd(const float* logits, float* P, int32_t* iters_out, int64_t n,
+                              int maxit, cudaStream_t s);
+cudaError_t launch_implicit_bwd(const float* logits, const float* P, const float* dP, float* dlogits,
+                                int64_t n, cudaStream_t s);
+
+cudaError_t launch_mix_fwd(const uint16_t* X, const float* H, const float* hpost, const uint16_t* F,
+                           uint16_t* Y, int64_t T, int64_t C, cudaStream_t s);
+cudaError_t launch_mix_bwd(const uint16_t* X, const float* H, const float* hpost, const uint16_t* F,
+                           const uint16_t* dY, uint16_t* dX, float* dH, float* dhpost, uint16_t* dF,
+                           float* dlogits, int64_t T, int64_t C, cudaStream_t s);
+cudaError_t launch_proj_mix_fwd(const float* logits, const float* hpost, const uint16_t* X,
+                                const uint16_t* F, uint16_t* Y, float* H, int64_t T, int64_t C,
+                                int maxit, cudaStream_t s);
+
+}  // namespace mhc

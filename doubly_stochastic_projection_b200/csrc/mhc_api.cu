@@ -1,0 +1,163 @@
+// mhc_api.cu -- the extern "C" entry points declared in include/mhc_birkhoff.h.
+//
+// Every entry point validates its arguments on the host (null pointers,
+// 16-byte alignment, sizes, method and iteration count) before enqueuing
+// anything, then launches on the caller's stream and returns immediately.
+#include <cstdint>
+
+#include "birkhoff_math.cuh"
+#include "launch.h"
+#include "mhc_birkhoff.h"
+
+namespace {
+
+constexpr int64_t kMaxC = int64_t(1) << 24;          // channels per stream
+constexpr int64_t kMaxElems = int64_t(1) << 40;      // bf16 elements per tensor
+
+bool misaligned(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MHC_OK : MHC_ERR_CUDA; }
+
+int check_matrices(int64_t n_mats)
+{
+    if (n_mats < 0 || n_mats > (int64_t(1) << 36)) return MHC_ERR_SIZE;
+    return MHC_OK;
+}
+
+int check_mix_sizes(int64_t T, int64_t C)
+{
+    if (T < 0 || C <= 0 || (C % 8) != 0 || C > kMaxC) return MHC_ERR_SIZE;
+    if (T > 0 && T * 4 > kMaxElems / C) return MHC_ERR_SIZE;
+    return MHC_OK;
+}
+
+int resolve_iters(int method, int iters, int* out)
+{
+    if (iters < 0 || iters > MHC_MAX_ITERS) return MHC_ERR_ARG;
+    if (method == MHC_SINKHORN)
+        *out = iters == 0 ? mhc::kDefaultSinkhornIters : iters;
+    else if (method == MHC_NEWTON)
+        *out = iters == 0 ? mhc::kDefaultNewtonIters : iters;
+    else
+        return MHC_ERR_ARG;
+    return MHC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mhc_version(void) { return 100; }
+
+const char* mhc_status_string(int status)
+{
+    switch (status) {
+    case MHC_OK: return "MHC_OK";
+    case MHC_ERR_NULL: return "MHC_ERR_NULL: a required pointer is NULL";
+    case MHC_ERR_ALIGN: return "MHC_ERR_ALIGN: a pointer is not 16-byte aligned";
+    case MHC_ERR_SIZE: return "MHC_ERR_SIZE: negative or unsupported size (C must be a positive multiple of 8)";
+    case MHC_ERR_ARG: return "MHC_ERR_ARG: unknown method or iteration count out of range";
+    case MHC_ERR_CUDA: return "MHC_ERR_CUDA: the CUDA runtime reported a launch error";
+    default: return "unknown mhc status";
+    }
+}
+
+int mhc_birkhoff_fwd(const float* logits, float* P, int64_t n_mats, int method, int iters, void* stream)
+{
+    int rc = check_matrices(n_mats);
+    if (rc != MHC_OK) return rc;
+    int it = 0;
+    if ((rc = resolve_iters(method, iters, &it)) != MHC_OK) return rc;
+    if (n_mats == 0) return MHC_OK;
+    if (!logits || !P) return MHC_ERR_NULL;
+    if (misaligned(logits) || misaligned(P)) return MHC_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (method == MHC_SINKHORN) return cuda_status(mhc::launch_sinkhorn_fwd(logits, P, n_mats, it, s));
+    return cuda_status(mhc::launch_newton_fwd(logits, P, nullptr, n_mats, it, s));
+}
+
+int mhc_birkhoff_fwd_diag(const float* logits, float* P, int32_t* iters_out, int64_t n_mats, int iters,
+                          void* stream)
+{
+    int rc = check_matrices(n_mats);
+    if (rc != MHC_OK) return rc;
+    int it = 0;
+    if ((rc = resolve_iters(MHC_NEWTON, iters, &it)) != MHC_OK) return rc;
+    if (n_mats == 0) return MHC_OK;
+    if (!logits || !P || !iters_out) return MHC_ERR_NULL;
+    if (misaligned(logits) || misaligned(P) || misaligned(iters_out)) return MHC_ERR_ALIGN;
+    return cuda_status(
+        mhc::launch_newton_fwd(logits, P, iters_out, n_mats, it, static_cast<cudaStream_t>(stream)));
+}
+
+int mhc_birkhoff_bwd(const float* logits, const float* P, const float* dP, float* dlogits, int64_t n_mats,
+                     void* stream)
+{
+    int rc = check_matrices(n_mats);
+    if (rc != MHC_OK) return rc;
+    if (n_mats == 0) return MHC_OK;
+    if (!dP || !dlogits || (!P && !logits)) return MHC_ERR_NULL;
+    if (misaligned(logits) || misaligned(P) || misaligned(dP) || misaligned(dlogits)) return MHC_ERR_ALIGN;
+    return cuda_status(
+        mhc::launch_implicit_bwd(logits, P, dP, dlogits, n_mats, static_cast<cudaStream_t>(stream)));
+}
+
+int mhc_residual_mix_fwd(const uint16_t* X, const float* H_res, const float* h_post, const uint16_t* F,
+                         uint16_t* Y, int64_t T, int64_t C, void* stream)
+{
+    int rc = check_mix_sizes(T, C);
+    if (rc != MHC_OK) return rc;
+    if (T == 0) return MHC_OK;
+    if (!X || !H_res || !h_post || !F || !Y) return MHC_ERR_NULL;
+    if (misaligned(X) || misaligned(H_res) || misaligned(h_post) || misaligned(F) || misaligned(Y))
+        return MHC_ERR_ALIGN;
+    return cuda_status(mhc::launch_mix_fwd(X, H_res, h_post, F, Y, T, C, static_cast<cudaStream_t>(stream)));
+}
+
+int mhc_residual_mix_bwd(const uint16_t* X, const float* H_res, const float* h_post, const uint16_t* F,
+                         const uint16_t* dY, uint16_t* dX, float* dH_res, float* dh_post, uint16_t* dF,
+                         float* dlogits, int64_t T, int64_t C, void* stream)
+{
+    int rc = check_mix_sizes(T, C);
+    if (rc != MHC_OK) return rc;
+    if (T == 0) return MHC_OK;
+    if (!X || !H_res || !h_post || !F || !dY || !dX || !dF) return MHC_ERR_NULL;
+    if (misaligned(X) || misaligned(H_res) || misaligned(h_post) || misaligned(F) || misaligned(dY) ||
+        misaligned(dX) || misaligned(dH_res) || misaligned(dh_post) || misaligned(dF) || misaligned(dlogits))
+        return MHC_ERR_ALIGN;
+    return cuda_status(mhc::launch_mix_bwd(X, H_res, h_post, F, dY, dX, dH_res, dh_post, dF, dlogits, T, C,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int mhc_proj_mix_fwd(const float* logits, const float* h_post, const uint16_t* X, const uint16_t* F,
+                     uint16_t* Y, float* H_res, int64_t T, int64_t C, int iters, void* stream)
+{
+    int rc = check_mix_sizes(T, C);
+    if (rc != MHC_OK) return rc;
+    int it = 0;
+    if ((rc = resolve_iters(MHC_NEWTON, iters, &it)) != MHC_OK) return rc;
+    if (T == 0) return MHC_OK;
+    if (!logits || !h_post || !X || !F || !Y || !H_res) return MHC_ERR_NULL;
+    if (misaligned(logits) || misaligned(h_post) || misaligned(X) || misaligned(F) || misaligned(Y) ||
+        misaligned(H_res))
+        return MHC_ERR_ALIGN;
+    return cuda_status(
+        mhc::launch_proj_mix_fwd(logits, h_post, X, F, Y, H_res, T, C, it, static_cast<cudaStream_t>(stream)));
+}
+
+int mhc_proj_mix_bwd(const float* H_res, const float* h_post, const uint16_t* X, const uint16_t* F,
+                     const uint16_t* dY, uint16_t* dX, float* dlogits, float* dh_post, uint16_t* dF, int64_t T,
+                     int64_t C, void* stream)
+{
+    int rc = check_mix_sizes(T, C);
+    if (rc != MHC_OK) return rc;
+    if (T == 0) return MHC_OK;
+    if (!H_res || !h_post || !X || !F || !dY || !dX || !dlogits || !dh_post || !dF) return MHC_ERR_NULL;
+    if (misaligned(H_res) || misaligned(h_post) || misaligned(X) || misaligned(F) || misaligned(dY) ||
+        misaligned(dX) || misaligned(dlogits) || misaligned(dh_post) || misaligned(dF))
+        return MHC_ERR_ALIGN;
+    return cuda_status(mhc::launch_mix_bwd(X, H_res, h_post, F, dY, dX, nullptr, dh_post, dF, dlogits, T, C,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

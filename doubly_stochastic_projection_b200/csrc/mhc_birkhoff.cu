@@ -1,0 +1,138 @@
+// mhc_birkhoff.cu -- batched 4x4 Birkhoff projection kernels for sm_100a.
+//
+// Layout choice: one thread per matrix.  The whole solve is register-resident
+// (16 floats of P plus a handful of scalars) and needs no cross-thread
+// communication, so no shuffle or shared-memory traffic is spent on column
+// sums; each thread reads its matrix as four 128-bit loads of whole rows and
+// writes it back the same way.  The warp-per-two-matrices, lane-per-entry
+// layout of the Birkhoff-acceleration summary (arXiv 2606.07574, §2.3) was
+// designed for an Ada GPU; here the projection is FP32/SFU-issue-bound
+// (Newton) or HBM-bound (backward), and a lane-per-entry layout would repeat
+// the 3x3 solve and the step logic on 16 lanes.
+#include <algorithm>
+#include <atomic>
+
+#include "birkhoff_math.cuh"
+#include "launch.h"
+
+namespace mhc {
+
+namespace {
+
+constexpr int kProjThreads = 256;
+
+__global__ void __launch_bounds__(kProjThreads)
+sinkhorn_fwd_kernel(const float* logits, float* P, int64_t n, int iters)
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
+        float a[16];
+        load16(logits + 16 * m, a);
+        sinkhorn_project(a, iters);
+        store16(P + 16 * m, a);
+    }
+}
+
+template <bool kDiag>
+__global__ void __launch_bounds__(kProjThreads)
+newton_fwd_kernel(const float* logits, float* P, int32_t* iters_out, int64_t n, int maxit)
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
+        float a[16];
+        load16(logits + 16 * m, a);
+        const int it = newton_project(a, maxit);
+        store16(P + 16 * m, a);
+        if (kDiag) iters_out[m] = it;
+    }
+}
+
+// kRecompute: P is not given; rebuild it from the logits by the Newton
+// forward before the backward (recompute instead of storing P).
+template <bool kRecompute>
+__global__ void __launch_bounds__(kProjThreads)
+implicit_bwd_kernel(const float* logits, const float* P, const float* dP, float* dlogits, int64_t n)
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
+        float p[16], g[16], out[16];
+        if (kRecompute) {
+            load16(logits + 16 * m, p);
+            newton_project(p, kDefaultNewtonIters);
+        } else {
+            load16(P + 16 * m, p);
+        }
+        load16(dP + 16 * m, g);
+        implicit_vjp(p, g, out);
+        store16(dlogits + 16 * m, out);
+    }
+}
+
+int64_t blocks_for(int64_t n, int threads) { return (n + threads - 1) / threads; }
+
+}  // namespace
+
+int device_sm_count()
+{
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 0 || dev >= 64) dev = 0;
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v <= 0) {
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+            v = 148;
+        cache[dev].store(v, std::memory_order_relaxed);
+    }
+    return v;
+}
+
+int persistent_grid(const void* kernel, int threads, size_t smem, int64_t blocks_needed)
+{
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess ||
+        per_sm <= 0)
+        per_sm = 1;
+    const int64_t full = (int64_t)per_sm * device_sm_count();
+    return (int)std::max<int64_t>(1, std::min<int64_t>(blocks_needed, full));
+}
+
+cudaError_t launch_sinkhorn_fwd(const float* logits, float* P, int64_t n, int iters, cudaStream_t s)
+{
+    const void* k = (const void*)sinkhorn_fwd_kernel;
+    const int grid = persistent_grid(k, kProjThreads, 0, blocks_for(n, kProjThreads));
+    sinkhorn_fwd_kernel<<<grid, kProjThreads, 0, s>>>(logits, P, n, iters);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_newton_fwd(const float* logits, float* P, int32_t* iters_out, int64_t n, int maxit,
+                              cudaStream_t s)
+{
+    if (iters_out) {
+        const int grid = persistent_grid((const void*)newton_fwd_kernel<true>, kProjThreads, 0,
+                                         blocks_for(n, kProjThreads));
+        newton_fwd_kernel<true><<<grid, kProjThreads, 0, s>>>(logits, P, iters_out, n, maxit);
+    } else {
+        const int grid = persistent_grid((const void*)newton_fwd_kernel<false>, kProjThreads, 0,
+                                         blocks_for(n, kProjThreads));
+        newton_fwd_kernel<false><<<grid, kProjThreads, 0, s>>>(logits, P, nullptr, n, maxit);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_implicit_bwd(const float* logits, const float* P, const float* dP, float* dlogits,
+                                int64_t n, cudaStream_t s)
+{
+    if (P) {
+        const int grid = persistent_grid((const void*)implicit_bwd_kernel<false>, kProjThreads, 0,
+                                         blocks_for(n, kProjThreads));
+        implicit_bwd_kernel<false><<<grid, kProjThreads, 0, s>>>(nullptr, P, dP, dlogits, n);
+    } else {
+        const int grid = persistent_grid((const void*)implicit_bwd_kernel<true>, kProjThreads, 0,
+                                         blocks_for(n, kProjThreads));
+        implicit_bwd_kernel<true><<<grid, kProjThreads, 0, s>>>(logits, nullptr, dP, dlogits, n);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace mhc

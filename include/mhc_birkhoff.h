@@ -52,6 +52,12 @@
 
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define MHC_API __attribute__((visibility("default")))
+#else
+#define MHC_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -100,7 +106,7 @@ enum mhc_method {
  *   iters   0 .. MHC_MAX_ITERS.
  *   stream  cudaStream_t or NULL.
  */
-int mhc_birkhoff_fwd(const float *logits, float *P, int64_t n_mats, int method, int iters,
+MHC_API int mhc_birkhoff_fwd(const float *logits, float *P, int64_t n_mats, int method, int iters,
                      void *stream);
 
 /*
@@ -111,7 +117,7 @@ int mhc_birkhoff_fwd(const float *logits, float *P, int64_t n_mats, int method, 
  *   iters_out [n_mats] int32, device, written.  Other arguments as
  *   mhc_birkhoff_fwd with method = MHC_NEWTON.
  */
-int mhc_birkhoff_fwd_diag(const float *logits, float *P, int32_t *iters_out, int64_t n_mats,
+MHC_API int mhc_birkhoff_fwd_diag(const float *logits, float *P, int32_t *iters_out, int64_t n_mats,
                           int iters, void *stream);
 
 /*
@@ -133,7 +139,7 @@ int mhc_birkhoff_fwd_diag(const float *logits, float *P, int32_t *iters_out, int
  *   dlogits  [n_mats][4][4] float, device, written.  May alias dP.
  *   At least one of logits and P must be non-NULL (MHC_ERR_NULL otherwise).
  */
-int mhc_birkhoff_bwd(const float *logits, const float *P, const float *dP, float *dlogits,
+MHC_API int mhc_birkhoff_bwd(const float *logits, const float *P, const float *dP, float *dlogits,
                      int64_t n_mats, void *stream);
 
 /*
@@ -149,7 +155,7 @@ int mhc_birkhoff_bwd(const float *logits, const float *P, const float *dP, float
  *   Y      [T][4][C] bf16, written (must not overlap X or F).
  *   T >= 0 tokens; C > 0, C % 8 == 0.
  */
-int mhc_residual_mix_fwd(const uint16_t *X, const float *H_res, const float *h_post,
+MHC_API int mhc_residual_mix_fwd(const uint16_t *X, const float *H_res, const float *h_post,
                          const uint16_t *F, uint16_t *Y, int64_t T, int64_t C, void *stream);
 
 /*
@@ -169,7 +175,7 @@ int mhc_residual_mix_fwd(const uint16_t *X, const float *H_res, const float *h_p
  *   dlogits [T][4][4] float, written, or NULL to skip.
  *   Reductions over C are accumulated in fp32.
  */
-int mhc_residual_mix_bwd(const uint16_t *X, const float *H_res, const float *h_post,
+MHC_API int mhc_residual_mix_bwd(const uint16_t *X, const float *H_res, const float *h_post,
                          const uint16_t *F, const uint16_t *dY, uint16_t *dX, float *dH_res,
                          float *dh_post, uint16_t *dF, float *dlogits, int64_t T, int64_t C,
                          void *stream);
@@ -182,7 +188,7 @@ int mhc_residual_mix_bwd(const uint16_t *X, const float *H_res, const float *h_p
  *   logits [T][4][4] float, read.    H_res [T][4][4] float, written.
  *   Other arguments as mhc_residual_mix_fwd.
  */
-int mhc_proj_mix_fwd(const float *logits, const float *h_post, const uint16_t *X,
+MHC_API int mhc_proj_mix_fwd(const float *logits, const float *h_post, const uint16_t *X,
                      const uint16_t *F, uint16_t *Y, float *H_res, int64_t T, int64_t C,
                      int iters, void *stream);
 
@@ -194,15 +200,15 @@ int mhc_proj_mix_fwd(const float *logits, const float *h_post, const uint16_t *X
  *   dlogits [T][4][4] float, written.  dh_post [T][4] float, written.
  *   dX, dF as in mhc_residual_mix_bwd.
  */
-int mhc_proj_mix_bwd(const float *H_res, const float *h_post, const uint16_t *X,
+MHC_API int mhc_proj_mix_bwd(const float *H_res, const float *h_post, const uint16_t *X,
                      const uint16_t *F, const uint16_t *dY, uint16_t *dX, float *dlogits,
                      float *dh_post, uint16_t *dF, int64_t T, int64_t C, void *stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
-const char *mhc_status_string(int status);
+MHC_API const char *mhc_status_string(int status);
 
 /* Library ABI version: major * 10000 + minor * 100 + patch. */
-int mhc_version(void);
+MHC_API int mhc_version(void);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,69 @@
+"""The C-ABI library builds for sm_100a, loads without a GPU, exports every
+symbol that include/mhc_birkhoff.h declares, and validates arguments on the
+host before touching CUDA.  No call here launches a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from doubly_stochastic_projection_b200 import build
+
+HEADER = os.path.join(build.ROOT, "include", "mhc_birkhoff.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MHC_API\s+[\w\s\*]*?\b(mhc_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("mhc_birkhoff_fwd", "mhc_birkhoff_bwd", "mhc_residual_mix_fwd", "mhc_residual_mix_bwd",
+              "mhc_proj_mix_fwd", "mhc_proj_mix_bwd", "mhc_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    import subprocess
+    out = subprocess.check_output(["nm", "-D", "--defined-only", build.LIB_PATH], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing
+    for n in _declared():
+        getattr(L, n)  # resolvable through the dynamic loader
+
+
+def test_host_only_calls(L):
+    L.mhc_status_string.restype = ctypes.c_char_p
+    L.mhc_status_string.argtypes = [ctypes.c_int]
+    assert L.mhc_status_string(0) == b"MHC_OK"
+    assert b"ALIGN" in L.mhc_status_string(2)
+    assert L.mhc_status_string(99) == b"unknown mhc status"
+    assert L.mhc_version() >= 100
+
+
+def test_validation_rejects_before_any_cuda_call(L):
+    p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    L.mhc_birkhoff_fwd.argtypes = [p, p, i64, i32, i32, p]
+    L.mhc_residual_mix_fwd.argtypes = [p, p, p, p, p, i64, i64, p]
+    L.mhc_birkhoff_bwd.argtypes = [p, p, p, p, i64, p]
+    fake = 1 << 20  # never dereferenced: every call below returns before launching
+    assert L.mhc_birkhoff_fwd(fake, fake, -5, 1, 0, None) == 3
+    assert L.mhc_birkhoff_fwd(fake, fake, 10, 2, 0, None) == 4
+    assert L.mhc_birkhoff_fwd(fake, fake, 10, 0, -1, None) == 4
+    assert L.mhc_birkhoff_fwd(fake, fake, 10, 1, 1001, None) == 4
+    assert L.mhc_birkhoff_fwd(None, fake, 10, 1, 0, None) == 1
+    assert L.mhc_birkhoff_fwd(fake + 4, fake, 10, 1, 0, None) == 2
+    assert L.mhc_birkhoff_fwd(None, None, 0, 1, 0, None) == 0      # empty batch: nothing to do
+    assert L.mhc_birkhoff_bwd(None, None, fake, fake, 3, None) == 1
+    assert L.mhc_residual_mix_fwd(fake, fake, fake, fake, fake, 4, 12, None) == 3
+    assert L.mhc_residual_mix_fwd(fake, fake, fake, fake, fake, 4, 0, None) == 3
+    assert L.mhc_residual_mix_fwd(fake, fake, fake, fake, fake + 8, 4, 16, None) == 2
+    assert L.mhc_residual_mix_fwd(None, None, None, None, None, 0, 16, None) == 0
