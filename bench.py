@@ -12,7 +12,7 @@ runs on the data path).
 Timing: W untimed warm-up steps; then, between a barrier and a device
 synchronisation on both sides, exactly K steps, each bracketed by CUDA events
 recorded on the stream the kernels run on, with the L2 cache flushed (a 512 MiB
-write) before every step and outside its events, because the step's 32 MiB
+read) before every step and outside its events, because the step's 32 MiB
 working set would otherwise stay in the 126 MB L2.  The reported time is the
 sum of the K step durations, maximised over ranks.
 
@@ -62,6 +62,14 @@ def parse():
     ap.add_argument("--no-extras", action="store_true", help="skip the sweep and mix extras")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-oracle sample budget")
+    ap.add_argument("--profile", default=None,
+                    choices=["newton_fwd", "sinkhorn_fwd", "implicit_bwd", "mix_fwd", "mix_bwd",
+                             "proj_mix_fwd", "proj_mix_bwd"],
+                    help="run one kernel --reps times on one case (for ncu) and exit")
+    ap.add_argument("--size", type=int, default=1 << 22, help="--profile: matrices, or tokens T for the mix")
+    ap.add_argument("--channels", type=int, default=4096, help="--profile: mix channels C")
+    ap.add_argument("--dist", default="normal1", help="--profile: logit distribution")
+    ap.add_argument("--reps", type=int, default=3)
     return ap.parse_args()
 
 
@@ -286,6 +294,8 @@ def event_time(fn, reps, stream, flush=None):
     """Mean device time (s) of fn() over reps, events on `stream`, flush outside."""
     import torch
 
+    fn()  # warm-up: allocator and first-launch costs stay outside the events
+    torch.cuda.synchronize()
     tot = 0.0
     for _ in range(reps):
         if flush is not None:
@@ -384,10 +394,13 @@ def run_b200(args):
     G = torch.from_numpy(G_np).to(dev)
     P = torch.empty_like(A)
     dl = torch.empty_like(A)
-    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_buf = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
     def flush():
-        flush_buf.zero_()
+        # a read of 4x the L2 size: evicts the previous step's lines and leaves
+        # L2 holding clean lines only, so no write-back of earlier data lands
+        # inside the next step's events
+        flush_buf.sum()
 
     def step():
         api.birkhoff_fwd(A, "newton", out=P)
@@ -422,6 +435,11 @@ def run_b200(args):
     t_max = max_over_ranks(t_step, pg, dev)
     value = world * N_MATS * K / t_max
     gpu_launches = 2 * K
+
+    _, its = api.birkhoff_fwd_diag(A)
+    itf = its.float()
+    newton_iters = {"mean": float(itf.mean()), "max": int(its.max()),
+                    "warp_max_mean": float(itf.reshape(-1, 32).max(1).values.mean())}
 
     # end to end through the public API, host buffers, copies timed
     A_h = A.cpu().pin_memory()
@@ -473,10 +491,11 @@ def run_b200(args):
         "config": {"workload": WORKLOAD, "n_mats_per_gpu": N_MATS,
                    "logits": "first half N(0,1), second half N(0,10^2), seed 2 (+7919*rank)",
                    "step": "Newton fwd (to max|colsum-1|<1e-6) + implicit bwd",
-                   "l2": "flushed (512 MiB write) before every step, outside its events",
+                   "l2": "flushed (512 MiB read) before every step, outside its events",
                    "parallelism": "token-sharded replicas, no collective" if world > 1 else "single GPU"},
         "fwd_matrices_per_s": world * N_MATS * K / max_over_ranks(t_fwd, pg, dev),
         "bwd_matrices_per_s": world * N_MATS * K / max_over_ranks(t_bwd, pg, dev),
+        "newton_iters": newton_iters,
         "e2e": e2e, "gpu_launches": gpu_launches, "roofline": roofline,
     }
 
@@ -507,8 +526,48 @@ def run_b200(args):
     return 0
 
 
+def run_profile_case(args):
+    """Run one kernel a few times on one case (for ncu captures)."""
+    import torch
+
+    from doubly_stochastic_projection_b200 import api, inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    k = args.profile
+    if k in ("newton_fwd", "sinkhorn_fwd", "implicit_bwd"):
+        n = args.size
+        A = torch.from_numpy(inputs.birkhoff_logits(n, args.dist, 5)).to(dev)
+        G = torch.from_numpy(inputs.upstream_grad(n, 6)).to(dev)
+        P = api.birkhoff_fwd(A, "newton")
+        out = torch.empty_like(A)
+        fn = {"newton_fwd": lambda: api.birkhoff_fwd(A, "newton", out=out),
+              "sinkhorn_fwd": lambda: api.birkhoff_fwd(A, "sinkhorn", 20, out=out),
+              "implicit_bwd": lambda: api.birkhoff_bwd(G, P=P, out=out)}[k]
+        desc = {"n_mats": n, "dist": args.dist}
+    else:
+        m = inputs.mix_workload("mix_T16384_C4096", device=dev, T=args.size, C=args.channels)
+        X, F, dY = m["X"], m["F"], m["dY"]
+        lg = torch.from_numpy(m["logits"]).to(dev)
+        h = torch.from_numpy(m["h_post"]).to(dev)
+        H = api.birkhoff_fwd(lg, "newton")
+        Y = torch.empty_like(X)
+        fn = {"mix_fwd": lambda: api.residual_mix_fwd(X, H, h, F, out=Y),
+              "mix_bwd": lambda: api.residual_mix_bwd(X, H, h, F, dY, need_dlogits=True),
+              "proj_mix_fwd": lambda: api.proj_mix_fwd(lg, h, X, F, out=Y, H_out=H),
+              "proj_mix_bwd": lambda: api.proj_mix_bwd(H, h, X, F, dY)}[k]
+        desc = {"T": args.size, "C": args.channels}
+    for _ in range(args.reps):
+        fn()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": k, "reps": args.reps, **desc}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    if args.profile:
+        return run_profile_case(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_b200(args)

@@ -301,44 +301,102 @@ __device__ __forceinline__ int newton_project(float (&a)[16], int maxit)
 //     J[X]_ik = P_ik sum_{j != k} P_ij (X_ik - X_ij),
 // which equals P_ik (X_ik - sum_j P_ij X_ij) for unit row sums but never
 // subtracts two nearly equal weighted means: for P close to a permutation
-// the weighted-mean form loses all relative accuracy in fp32.
+// the weighted-mean form loses all relative accuracy.
+//
+// The arithmetic is carried out in double precision (fp32 in, fp32 out).
+// For P close to a permutation the result is tiny and comes out of a
+// cancellation: G_ik - G_ij - (lambda_k - lambda_j) is many orders smaller
+// than its O(1) terms, so the fp32 rounding of lambda alone would cost up to
+// 1e-3 of the result's relative accuracy.  The backward reads and writes
+// 192 bytes per matrix against about 250 arithmetic operations, so on B200
+// (FP64 at half the FP32 rate) the extra width stays under the HBM time.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void implicit_vjp(const float (&p)[16], const float (&g)[16],
-                                             float (&out)[16])
+struct PairWeightsD {
+    double w01, w02, w03, w12, w13, w23;
+};
+
+__device__ __forceinline__ PairWeightsD pair_weights_d(const double (&p)[16])
 {
-    float D[4][6];
-    float c0 = 0.0f, c1 = 0.0f, c2 = 0.0f;
+    PairWeightsD w;
+    w.w01 = p[0] * p[1];
+    w.w02 = p[0] * p[2];
+    w.w03 = p[0] * p[3];
+    w.w12 = p[1] * p[2];
+    w.w13 = p[1] * p[3];
+    w.w23 = p[2] * p[3];
+#pragma unroll
+    for (int r = 1; r < 4; ++r) {
+        const double* q = p + 4 * r;
+        w.w01 = fma(q[0], q[1], w.w01);
+        w.w02 = fma(q[0], q[2], w.w02);
+        w.w03 = fma(q[0], q[3], w.w03);
+        w.w12 = fma(q[1], q[2], w.w12);
+        w.w13 = fma(q[1], q[3], w.w13);
+        w.w23 = fma(q[2], q[3], w.w23);
+    }
+    return w;
+}
+
+// Grounded-Laplacian solve in double precision (same elimination order as
+// laplacian_solve).
+__device__ __forceinline__ bool laplacian_solve_d(const PairWeightsD& w, double r0, double r1, double r2,
+                                                  double& x0, double& x1, double& x2)
+{
+    const double a = (w.w01 + w.w02) + w.w03;
+    const double ia = 1.0 / a;
+    const double v12 = fma(w.w01 * w.w02, ia, w.w12);
+    const double v13 = fma(w.w01 * w.w03, ia, w.w13);
+    const double v23 = fma(w.w02 * w.w03, ia, w.w23);
+    const double q1 = fma(w.w01 * r0, ia, r1);
+    const double q2 = fma(w.w02 * r0, ia, r2);
+    const double b = v12 + v13;
+    const double ib = 1.0 / b;
+    const double u = fma(v12 * v13, ib, v23);
+    const double q2b = fma(v12 * q1, ib, q2);
+    x2 = q2b / u;
+    x1 = fma(v12, x2, q1) * ib;
+    x0 = fma(w.w01, x1, fma(w.w02, x2, r0)) * ia;
+    return (a > 0.0) && (b > 0.0) && (u > 0.0) && isfinite(x0) && isfinite(x1) && isfinite(x2);
+}
+
+__device__ __forceinline__ void implicit_vjp(const float (&pf)[16], const float (&gf)[16], float (&out)[16])
+{
+    double p[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) p[k] = (double)pf[k];
+    double D[4][6];
+    double c0 = 0.0, c1 = 0.0, c2 = 0.0;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        const float* x = g + 4 * r;
-        const float* q = p + 4 * r;
-        D[r][0] = x[0] - x[1];
-        D[r][1] = x[0] - x[2];
-        D[r][2] = x[0] - x[3];
-        D[r][3] = x[1] - x[2];
-        D[r][4] = x[1] - x[3];
-        D[r][5] = x[2] - x[3];
-        c0 = fmaf(q[0], fmaf(q[1], D[r][0], fmaf(q[2], D[r][1], q[3] * D[r][2])), c0);
-        c1 = fmaf(q[1], fmaf(q[2], D[r][3], fmaf(q[3], D[r][4], -q[0] * D[r][0])), c1);
-        c2 = fmaf(q[2], fmaf(q[3], D[r][5], fmaf(-q[0], D[r][1], -q[1] * D[r][3])), c2);
+        const double x0 = gf[4 * r], x1 = gf[4 * r + 1], x2 = gf[4 * r + 2], x3 = gf[4 * r + 3];
+        const double* q = p + 4 * r;
+        D[r][0] = x0 - x1;
+        D[r][1] = x0 - x2;
+        D[r][2] = x0 - x3;
+        D[r][3] = x1 - x2;
+        D[r][4] = x1 - x3;
+        D[r][5] = x2 - x3;
+        c0 = fma(q[0], fma(q[1], D[r][0], fma(q[2], D[r][1], q[3] * D[r][2])), c0);
+        c1 = fma(q[1], fma(q[2], D[r][3], fma(q[3], D[r][4], -q[0] * D[r][0])), c1);
+        c2 = fma(q[2], fma(q[3], D[r][5], fma(-q[0], D[r][1], -q[1] * D[r][3])), c2);
     }
-    float l0, l1, l2;
-    const bool ok = laplacian_solve(pair_weights(p), c0, c1, c2, l0, l1, l2);
+    double l0, l1, l2;
+    const bool ok = laplacian_solve_d(pair_weights_d(p), c0, c1, c2, l0, l1, l2);
     if (!ok) {
         fill_nan(out);
         return;
     }
-    const float L[6] = {l0 - l1, l0 - l2, l0, l1 - l2, l1, l2};
+    const double L[6] = {l0 - l1, l0 - l2, l0, l1 - l2, l1, l2};
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        const float* q = p + 4 * r;
-        float E[6];
+        const double* q = p + 4 * r;
+        double E[6];
 #pragma unroll
         for (int k = 0; k < 6; ++k) E[k] = D[r][k] - L[k];
-        out[4 * r + 0] = q[0] * fmaf(q[1], E[0], fmaf(q[2], E[1], q[3] * E[2]));
-        out[4 * r + 1] = q[1] * fmaf(q[2], E[3], fmaf(q[3], E[4], -q[0] * E[0]));
-        out[4 * r + 2] = q[2] * fmaf(q[3], E[5], fmaf(-q[0], E[1], -q[1] * E[3]));
-        out[4 * r + 3] = q[3] * fmaf(-q[0], E[2], fmaf(-q[1], E[4], -q[2] * E[5]));
+        out[4 * r + 0] = (float)(q[0] * fma(q[1], E[0], fma(q[2], E[1], q[3] * E[2])));
+        out[4 * r + 1] = (float)(q[1] * fma(q[2], E[3], fma(q[3], E[4], -q[0] * E[0])));
+        out[4 * r + 2] = (float)(q[2] * fma(q[3], E[5], fma(-q[0], E[1], -q[1] * E[3])));
+        out[4 * r + 3] = (float)(q[3] * fma(-q[0], E[2], fma(-q[1], E[4], -q[2] * E[5])));
     }
 }
 
