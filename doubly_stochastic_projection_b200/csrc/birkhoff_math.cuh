@@ -17,7 +17,7 @@
 
 namespace mhc {
 
-constexpr int kDefaultNewtonIters = 30;
+constexpr int kDefaultNewtonIters = 50;
 constexpr int kDefaultSinkhornIters = 20;
 // Newton stops once every column sum is within this of one (rows are
 // normalised exactly, up to rounding, at every iterate).
@@ -27,10 +27,21 @@ constexpr float kNewtonTol = 1e-6f;
 constexpr float kLineSearchAbove = 1e-2f;
 constexpr float kArmijo = 1e-4f;
 constexpr int kMaxHalvings = 24;
-// No dual potential moves by more than this (in log units) per iteration.
-constexpr float kStepCap = 16.0f;
+// No dual potential moves by more than this (in log units) per iteration.  A
+// longer cap (16) let capped steps along a nearly singular Hessian direction
+// zigzag for ever on about 3 in 10^6 N(0, 10^2) matrices.
+constexpr float kStepCap = 4.0f;
 
-__device__ __forceinline__ float rcp_rn(float x) { return __frcp_rn(x); }
+// Reciprocal to within 1 ulp (MUFU), flushing subnormals.  Used where a
+// reciprocal only rescales an iterate (normalisations, elimination pivots):
+// the next iterate is renormalised and convergence is judged on it, so the
+// last-bit rounding of the scale cannot move the fixed point.
+__device__ __forceinline__ float rcp_approx(float x)
+{
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 __device__ __forceinline__ void load16(const float* p, float (&a)[16])
 {
@@ -58,7 +69,7 @@ __device__ __forceinline__ void normalize_rows(float (&a)[16])
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         const float s = (a[4 * r] + a[4 * r + 1]) + (a[4 * r + 2] + a[4 * r + 3]);
-        const float q = rcp_rn(s);
+        const float q = rcp_approx(s);
 #pragma unroll
         for (int c = 0; c < 4; ++c) a[4 * r + c] *= q;
     }
@@ -69,7 +80,7 @@ __device__ __forceinline__ void normalize_cols(float (&a)[16])
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
         const float s = (a[c] + a[4 + c]) + (a[8 + c] + a[12 + c]);
-        const float q = rcp_rn(s);
+        const float q = rcp_approx(s);
 #pragma unroll
         for (int r = 0; r < 4; ++r) a[4 * r + c] *= q;
     }
@@ -93,14 +104,6 @@ __device__ __forceinline__ void shift_cols_by_max(float (&a)[16])
 #pragma unroll
         for (int r = 0; r < 4; ++r) a[4 * r + c] -= m;
     }
-}
-
-__device__ __forceinline__ bool all_finite(const float (&a)[16])
-{
-    bool ok = true;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) ok = ok && isfinite(a[k]);
-    return ok;
 }
 
 __device__ __forceinline__ void fill_nan(float (&a)[16])
@@ -154,7 +157,7 @@ __device__ __forceinline__ bool laplacian_solve(const PairWeights& w, float r0, 
                                                 float& x0, float& x1, float& x2)
 {
     const float a = (w.w01 + w.w02) + w.w03;
-    const float ia = rcp_rn(a);
+    const float ia = rcp_approx(a);
     // eliminate node 0: reduced weights among nodes 1, 2 and ground
     const float v12 = fmaf(w.w01 * w.w02, ia, w.w12);
     const float v13 = fmaf(w.w01 * w.w03, ia, w.w13);
@@ -163,15 +166,15 @@ __device__ __forceinline__ bool laplacian_solve(const PairWeights& w, float r0, 
     const float q2 = fmaf(w.w02 * r0, ia, r2);
     // eliminate node 1
     const float b = v12 + v13;
-    const float ib = rcp_rn(b);
+    const float ib = rcp_approx(b);
     const float u = fmaf(v12 * v13, ib, v23);
     const float q2b = fmaf(v12 * q1, ib, q2);
-    x2 = q2b * rcp_rn(u);
+    x2 = q2b * rcp_approx(u);
     x1 = fmaf(v12, x2, q1) * ib;
     x0 = fmaf(w.w01, x1, fmaf(w.w02, x2, r0)) * ia;
-    const bool piv = (a > 0.0f) && (b > 0.0f) && (u > 0.0f) && (ia <= 3.0e38f) &&
-                     (ib <= 3.0e38f);
-    return piv && isfinite(x0) && isfinite(x1) && isfinite(x2);
+    // positive pivots and a finite solution (x0 + x1 + x2 is non-finite if
+    // any component is)
+    return (a > 0.0f) && (b > 0.0f) && (u > 0.0f) && isfinite((x0 + x1) + x2);
 }
 
 // ---------------------------------------------------------------------------
@@ -204,26 +207,23 @@ __device__ __forceinline__ void sinkhorn_project(float (&a)[16], int iters)
 // same map as g += t d but keeps every entry in [0, 1] and needs three exps
 // per step instead of sixteen.  Start: A shifted by its row maxima and then
 // its column maxima (P is unchanged by either, [BA] §2.1 shift redundancy and
-// max shift), exponentiated, rows normalised, then one Sinkhorn round as a
-// warm start.  Globalisation: the step is capped at kStepCap per potential,
+// max shift), exponentiated, then one Sinkhorn round as a warm start.  Globalisation: the step is capped at kStepCap per potential,
 // Armijo backtracking on phi while the error is large; a Sinkhorn round
 // replaces the step when the Laplacian is singular or no decrease is found.
 // Returns the number of Newton iterations taken.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int newton_project(float (&a)[16], int maxit)
 {
-    if (!all_finite(a)) {
-        fill_nan(a);
-        return 0;
-    }
     shift_rows_by_max(a);
     shift_cols_by_max(a);
 #pragma unroll
     for (int k = 0; k < 16; ++k) a[k] = expf(a[k]);
-    normalize_rows(a);
+    // one Sinkhorn round (columns, then rows) as the warm start; every row and
+    // column of exp(A) now holds a 1, so no sum is below one
     normalize_cols(a);
     normalize_rows(a);
 
+    float err = 0.0f;
     int it = 0;
     for (; it < maxit; ++it) {
         const float c0 = (a[0] + a[4]) + (a[8] + a[12]);
@@ -231,63 +231,64 @@ __device__ __forceinline__ int newton_project(float (&a)[16], int maxit)
         const float c2 = (a[2] + a[6]) + (a[10] + a[14]);
         const float c3 = (a[3] + a[7]) + (a[11] + a[15]);
         const float g0 = c0 - 1.0f, g1 = c1 - 1.0f, g2 = c2 - 1.0f;
-        const float err = fmaxf(fmaxf(fabsf(g0), fabsf(g1)), fmaxf(fabsf(g2), fabsf(c3 - 1.0f)));
-        if (!(err >= kNewtonTol)) break;
+        err = fmaxf(fmaxf(fabsf(g0), fabsf(g1)), fmaxf(fabsf(g2), fabsf(c3 - 1.0f)));
+        if (!(err >= kNewtonTol)) break;  // converged, or NaN from a non-finite input
 
         const PairWeights w = pair_weights(a);
         float d0, d1, d2;
         bool ok = laplacian_solve(w, -g0, -g1, -g2, d0, d1, d2);
         const float dmax = fmaxf(fmaxf(fabsf(d0), fabsf(d1)), fabsf(d2));
-        if (ok && dmax > kStepCap) {
-            const float s = kStepCap / dmax;
-            d0 *= s;
-            d1 *= s;
-            d2 *= s;
+        if (dmax > kStepCap) {
+            const float sc = kStepCap * rcp_approx(dmax);
+            d0 *= sc;
+            d1 *= sc;
+            d2 *= sc;
         }
-        float e0 = 1.0f, e1 = 1.0f, e2 = 1.0f;
-        if (ok) {
-            e0 = expf(d0);
-            e1 = expf(d1);
-            e2 = expf(d2);
-            if (err >= kLineSearchAbove) {
-                // phi(g + t d) - phi(g) = sum_i log(sum_j P_ij e^{t d_j}) - t sum_j d_j
-                const float slope = fmaf(g0, d0, fmaf(g1, d1, g2 * d2));
-                const float dsum = (d0 + d1) + d2;
-                float t = 1.0f;
-                ok = false;
-                for (int h = 0; h < kMaxHalvings && slope < 0.0f; ++h) {
-                    float prod = 1.0f;
+        // Column factors e^{t d_j}.  Their rounding only perturbs the step,
+        // never the fixed point, so the fast exponential is used here (the
+        // exponential of the logits above is the exact one).
+        float e0 = __expf(d0), e1 = __expf(d1), e2 = __expf(d2);
+        float s[4];
 #pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        const float s =
-                            fmaf(a[4 * r], e0, fmaf(a[4 * r + 1], e1, fmaf(a[4 * r + 2], e2, a[4 * r + 3])));
-                        prod *= s;
-                    }
-                    const float dphi = logf(prod) - t * dsum;
-                    if (dphi <= kArmijo * t * slope) {
-                        ok = true;
-                        break;
-                    }
-                    t *= 0.5f;
-                    e0 = expf(t * d0);
-                    e1 = expf(t * d1);
-                    e2 = expf(t * d2);
+        for (int r = 0; r < 4; ++r)
+            s[r] = fmaf(a[4 * r], e0, fmaf(a[4 * r + 1], e1, fmaf(a[4 * r + 2], e2, a[4 * r + 3])));
+        if (ok && err >= kLineSearchAbove) {
+            // Armijo on phi: phi(g + t d) - phi(g) = sum_i log(sum_j P_ij e^{t d_j}) - t sum_j d_j
+            const float slope = fmaf(g0, d0, fmaf(g1, d1, g2 * d2));
+            const float dsum = (d0 + d1) + d2;
+            float t = 1.0f;
+            ok = false;
+            for (int h = 0; h < kMaxHalvings && slope < 0.0f; ++h) {
+                const float dphi = __logf((s[0] * s[1]) * (s[2] * s[3])) - t * dsum;
+                if (dphi <= kArmijo * t * slope) {
+                    ok = true;
+                    break;
                 }
+                t *= 0.5f;
+                e0 = __expf(t * d0);
+                e1 = __expf(t * d1);
+                e2 = __expf(t * d2);
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+                    s[r] = fmaf(a[4 * r], e0, fmaf(a[4 * r + 1], e1, fmaf(a[4 * r + 2], e2, a[4 * r + 3])));
             }
         }
         if (ok) {
+            // P_ij <- P_ij e^{t d_j} / s_i
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
-                a[4 * r + 0] *= e0;
-                a[4 * r + 1] *= e1;
-                a[4 * r + 2] *= e2;
+                const float q = rcp_approx(s[r]);
+                a[4 * r + 0] *= e0 * q;
+                a[4 * r + 1] *= e1 * q;
+                a[4 * r + 2] *= e2 * q;
+                a[4 * r + 3] *= q;
             }
-            normalize_rows(a);
         } else {
             normalize_cols(a);
             normalize_rows(a);
         }
     }
+    if (err != err) fill_nan(a);  // a non-finite logit poisons its whole matrix
     return it;
 }
 
