@@ -31,6 +31,8 @@ constexpr int kMaxHalvings = 24;
 // longer cap (16) let capped steps along a nearly singular Hessian direction
 // zigzag for ever on about 3 in 10^6 N(0, 10^2) matrices.
 constexpr float kStepCap = 4.0f;
+// Levenberg-Marquardt damping factor (see newton_project).
+constexpr float kDamping = 0.03f;
 
 // Reciprocal to within 1 ulp (MUFU), flushing subnormals.  Used where a
 // reciprocal only rescales an iterate (normalisations, elimination pivots):
@@ -196,6 +198,66 @@ __device__ __forceinline__ void sinkhorn_project(float (&a)[16], int iters)
 }
 
 // ---------------------------------------------------------------------------
+// Relative-accuracy polish for matrices close to a permutation.
+//
+// In fp32, colsum_j - 1 for a column whose largest entry is ~1 carries the
+// rounding of that entry (~6e-8), so Newton stops with the small entries of
+// such a matrix accurate only in absolute terms: entries of 1e-4 are then off
+// by up to 1e-3 of their value, and so is the gradient, which scales with
+// them.  When every row has an entry >= 0.9 (at convergence these sit in
+// distinct columns, as each column sums to one), the deviation can instead be
+// formed from small numbers only, taking each row's dominant entry as one
+// minus the rest of its row:
+//     colsum_j - 1 = sum_{i: k_i != j} P_ij - sum_{k != j} P_{i*,k},
+// where i* is the row whose dominant entry is in column j.  One Newton step on
+// this gradient (quadratic convergence from ~1e-3 relative error) leaves the
+// small entries accurate to about 1e-7 of their value.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void polish_near_permutation(float (&a)[16])
+{
+    float m[4];
+    int k[4];
+    unsigned cols = 0;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const float* q = a + 4 * r;
+        m[r] = fmaxf(fmaxf(q[0], q[1]), fmaxf(q[2], q[3]));
+        k[r] = q[0] == m[r] ? 0 : q[1] == m[r] ? 1 : q[2] == m[r] ? 2 : 3;
+        cols |= 1u << k[r];
+    }
+    if (fminf(fminf(m[0], m[1]), fminf(m[2], m[3])) < 0.9f || cols != 15u) return;
+    // off-dominant mass of each row, summed without its dominant entry
+    float o[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const float* q = a + 4 * r;
+        o[r] = ((k[r] == 0 ? 0.0f : q[0]) + (k[r] == 1 ? 0.0f : q[1])) +
+               ((k[r] == 2 ? 0.0f : q[2]) + (k[r] == 3 ? 0.0f : q[3]));
+    }
+    float g[3];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        float sum = 0.0f;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) sum += k[r] == j ? -o[r] : a[4 * r + j];
+        g[j] = sum;
+    }
+    const PairWeights w = pair_weights(a);
+    float d0, d1, d2;
+    if (!laplacian_solve(w, -g[0], -g[1], -g[2], d0, d1, d2)) return;
+    const float e0 = __expf(d0), e1 = __expf(d1), e2 = __expf(d2);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const float sr = fmaf(a[4 * r], e0, fmaf(a[4 * r + 1], e1, fmaf(a[4 * r + 2], e2, a[4 * r + 3])));
+        const float q = rcp_approx(sr);
+        a[4 * r + 0] *= e0 * q;
+        a[4 * r + 1] *= e1 * q;
+        a[4 * r + 2] *= e2 * q;
+        a[4 * r + 3] *= q;
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Forward solver 2: Newton's method on the 3-variable reduced dual ([BA] §2,
 // §2.1).  The projection is P_ij = exp(A_ij + f_i + g_j) with unit row and
 // column sums.  Eliminating f leaves the convex
@@ -207,10 +269,14 @@ __device__ __forceinline__ void sinkhorn_project(float (&a)[16], int iters)
 // same map as g += t d but keeps every entry in [0, 1] and needs three exps
 // per step instead of sixteen.  Start: A shifted by its row maxima and then
 // its column maxima (P is unchanged by either, [BA] §2.1 shift redundancy and
-// max shift), exponentiated, then one Sinkhorn round as a warm start.  Globalisation: the step is capped at kStepCap per potential,
+// max shift), exponentiated, then one Sinkhorn round as a warm start.
+// Globalisation (the pages give none): Levenberg-Marquardt damping
+// proportional to the error, the step capped at kStepCap per potential, and
 // Armijo backtracking on phi while the error is large; a Sinkhorn round
 // replaces the step when the Laplacian is singular or no decrease is found.
-// Returns the number of Newton iterations taken.
+// After convergence, matrices close to a permutation get one more step with
+// a cancellation-free gradient (polish_near_permutation).
+// Returns the number of Newton iterations taken (the polish step not counted).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ int newton_project(float (&a)[16], int maxit)
 {
@@ -234,7 +300,18 @@ __device__ __forceinline__ int newton_project(float (&a)[16], int maxit)
         err = fmaxf(fmaxf(fabsf(g0), fabsf(g1)), fmaxf(fabsf(g2), fabsf(c3 - 1.0f)));
         if (!(err >= kNewtonTol)) break;  // converged, or NaN from a non-finite input
 
-        const PairWeights w = pair_weights(a);
+        // Levenberg-Marquardt damping: solve (H + mu I) d = -grad with
+        // mu = kDamping * err * mean(diag H).  Adding mu I to the grounded
+        // Laplacian is adding mu to each column's edge to ground, so the
+        // elimination below stays cancellation-free.  The damping shortens the
+        // step along nearly singular Hessian directions, where undamped
+        // capped Newton steps can zigzag without converging, and vanishes
+        // with err, keeping the quadratic end-game.
+        PairWeights w = pair_weights(a);
+        const float mu = kDamping * err * ((w.w03 + w.w13 + w.w23) + 2.0f * ((w.w01 + w.w02) + w.w12)) * (1.0f / 3.0f);
+        w.w03 += mu;
+        w.w13 += mu;
+        w.w23 += mu;
         float d0, d1, d2;
         bool ok = laplacian_solve(w, -g0, -g1, -g2, d0, d1, d2);
         const float dmax = fmaxf(fmaxf(fabsf(d0), fabsf(d1)), fabsf(d2));
@@ -288,7 +365,10 @@ __device__ __forceinline__ int newton_project(float (&a)[16], int maxit)
             normalize_rows(a);
         }
     }
-    if (err != err) fill_nan(a);  // a non-finite logit poisons its whole matrix
+    if (err != err)
+        fill_nan(a);  // a non-finite logit poisons its whole matrix
+    else if (err < kNewtonTol)
+        polish_near_permutation(a);
     return it;
 }
 
@@ -316,24 +396,18 @@ struct PairWeightsD {
     double w01, w02, w03, w12, w13, w23;
 };
 
-__device__ __forceinline__ PairWeightsD pair_weights_d(const double (&p)[16])
+__device__ __forceinline__ PairWeightsD pair_weights_d(const float (&p)[16])
 {
-    PairWeightsD w;
-    w.w01 = p[0] * p[1];
-    w.w02 = p[0] * p[2];
-    w.w03 = p[0] * p[3];
-    w.w12 = p[1] * p[2];
-    w.w13 = p[1] * p[3];
-    w.w23 = p[2] * p[3];
+    PairWeightsD w = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-    for (int r = 1; r < 4; ++r) {
-        const double* q = p + 4 * r;
-        w.w01 = fma(q[0], q[1], w.w01);
-        w.w02 = fma(q[0], q[2], w.w02);
-        w.w03 = fma(q[0], q[3], w.w03);
-        w.w12 = fma(q[1], q[2], w.w12);
-        w.w13 = fma(q[1], q[3], w.w13);
-        w.w23 = fma(q[2], q[3], w.w23);
+    for (int r = 0; r < 4; ++r) {
+        const double q0 = p[4 * r], q1 = p[4 * r + 1], q2 = p[4 * r + 2], q3 = p[4 * r + 3];
+        w.w01 = fma(q0, q1, w.w01);
+        w.w02 = fma(q0, q2, w.w02);
+        w.w03 = fma(q0, q3, w.w03);
+        w.w12 = fma(q1, q2, w.w12);
+        w.w13 = fma(q1, q3, w.w13);
+        w.w23 = fma(q2, q3, w.w23);
     }
     return w;
 }
@@ -360,44 +434,51 @@ __device__ __forceinline__ bool laplacian_solve_d(const PairWeightsD& w, double 
     return (a > 0.0) && (b > 0.0) && (u > 0.0) && isfinite(x0) && isfinite(x1) && isfinite(x2);
 }
 
+// Pairwise differences of one row of X, in double (exact for fp32 inputs):
+// D = {x0-x1, x0-x2, x0-x3, x1-x2, x1-x3, x2-x3}.
+__device__ __forceinline__ void row_differences(const float* x, double (&D)[6])
+{
+    const double x0 = x[0], x1 = x[1], x2 = x[2], x3 = x[3];
+    D[0] = x0 - x1;
+    D[1] = x0 - x2;
+    D[2] = x0 - x3;
+    D[3] = x1 - x2;
+    D[4] = x1 - x3;
+    D[5] = x2 - x3;
+}
+
 __device__ __forceinline__ void implicit_vjp(const float (&pf)[16], const float (&gf)[16], float (&out)[16])
 {
-    double p[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) p[k] = (double)pf[k];
-    double D[4][6];
+    // pass 1: column sums of S = J[G] (columns 0..2)
     double c0 = 0.0, c1 = 0.0, c2 = 0.0;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        const double x0 = gf[4 * r], x1 = gf[4 * r + 1], x2 = gf[4 * r + 2], x3 = gf[4 * r + 3];
-        const double* q = p + 4 * r;
-        D[r][0] = x0 - x1;
-        D[r][1] = x0 - x2;
-        D[r][2] = x0 - x3;
-        D[r][3] = x1 - x2;
-        D[r][4] = x1 - x3;
-        D[r][5] = x2 - x3;
-        c0 = fma(q[0], fma(q[1], D[r][0], fma(q[2], D[r][1], q[3] * D[r][2])), c0);
-        c1 = fma(q[1], fma(q[2], D[r][3], fma(q[3], D[r][4], -q[0] * D[r][0])), c1);
-        c2 = fma(q[2], fma(q[3], D[r][5], fma(-q[0], D[r][1], -q[1] * D[r][3])), c2);
+        double D[6];
+        row_differences(gf + 4 * r, D);
+        const double q0 = pf[4 * r], q1 = pf[4 * r + 1], q2 = pf[4 * r + 2], q3 = pf[4 * r + 3];
+        c0 = fma(q0, fma(q1, D[0], fma(q2, D[1], q3 * D[2])), c0);
+        c1 = fma(q1, fma(q2, D[3], fma(q3, D[4], -q0 * D[0])), c1);
+        c2 = fma(q2, fma(q3, D[5], fma(-q0, D[1], -q1 * D[3])), c2);
     }
     double l0, l1, l2;
-    const bool ok = laplacian_solve_d(pair_weights_d(p), c0, c1, c2, l0, l1, l2);
+    const bool ok = laplacian_solve_d(pair_weights_d(pf), c0, c1, c2, l0, l1, l2);
     if (!ok) {
         fill_nan(out);
         return;
     }
     const double L[6] = {l0 - l1, l0 - l2, l0, l1 - l2, l1, l2};
+    // pass 2: J[G - 1 lambda^T], differences recomputed rather than kept
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        const double* q = p + 4 * r;
         double E[6];
+        row_differences(gf + 4 * r, E);
 #pragma unroll
-        for (int k = 0; k < 6; ++k) E[k] = D[r][k] - L[k];
-        out[4 * r + 0] = (float)(q[0] * fma(q[1], E[0], fma(q[2], E[1], q[3] * E[2])));
-        out[4 * r + 1] = (float)(q[1] * fma(q[2], E[3], fma(q[3], E[4], -q[0] * E[0])));
-        out[4 * r + 2] = (float)(q[2] * fma(q[3], E[5], fma(-q[0], E[1], -q[1] * E[3])));
-        out[4 * r + 3] = (float)(q[3] * fma(-q[0], E[2], fma(-q[1], E[4], -q[2] * E[5])));
+        for (int k = 0; k < 6; ++k) E[k] -= L[k];
+        const double q0 = pf[4 * r], q1 = pf[4 * r + 1], q2 = pf[4 * r + 2], q3 = pf[4 * r + 3];
+        out[4 * r + 0] = (float)(q0 * fma(q1, E[0], fma(q2, E[1], q3 * E[2])));
+        out[4 * r + 1] = (float)(q1 * fma(q2, E[3], fma(q3, E[4], -q0 * E[0])));
+        out[4 * r + 2] = (float)(q2 * fma(q3, E[5], fma(-q0, E[1], -q1 * E[3])));
+        out[4 * r + 3] = (float)(q3 * fma(-q0, E[2], fma(-q1, E[4], -q2 * E[5])));
     }
 }
 

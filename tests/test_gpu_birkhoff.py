@@ -93,10 +93,15 @@ def test_end_to_end_gradient_against_oracle_projection(orc):
         P_g = api.birkhoff_fwd(to_gpu(A), "newton")
         dl = to_np64(api.birkhoff_bwd(to_gpu(G), P=P_g))
         ref = orc.implicit_bwd(orc.newton(A.astype(np.float64), tol=1e-13, max_iter=200), G.astype(np.float64))
-        rel, _ = per_matrix_rel_err(dl, ref)
+        rel, scale = per_matrix_rel_err(dl, ref)
         assert np.median(rel) <= GRAD_REL_TOL, (dist, np.median(rel))
+        # batch-normalised: every entry within 1e-4 of the largest gradient
         assert np.abs(dl - ref).max() <= GRAD_REL_TOL * np.abs(ref).max(), dist
-        assert rel.max() <= 5e-2, (dist, rel.max())
+        # per matrix, wherever the gradient is not itself at the scale of the
+        # forward's absolute error
+        big = scale >= 1e-2 * np.abs(G).reshape(-1, 16).max(1)
+        assert big.mean() > 0.5
+        assert rel[big].max() <= 1e-3, (dist, rel[big].max())
 
 
 @pytest.mark.parametrize("si", range(len(inputs.SWEEP_SIZES)))
