@@ -325,6 +325,7 @@ def extras(dev, stream, flush, hbm, api, inputs):
             api.birkhoff_fwd(A, "newton", out=P)
             _, its = api.birkhoff_fwd_diag(A)
             tf = event_time(lambda: api.birkhoff_fwd(A, "newton", out=P), reps, stream, flush)
+            tr = event_time(lambda: api.birkhoff_fwd(A, "newton_refined", out=dl), reps, stream, flush)
             tb = event_time(lambda: api.birkhoff_bwd(G, P=P, out=dl), reps, stream, flush)
             itn = its.float()
             out["sweep"].append({
@@ -333,6 +334,7 @@ def extras(dev, stream, flush, hbm, api, inputs):
                 "fwd_gbs": BYTES_FWD * n / tf / 1e9, "bwd_gbs": BYTES_BWD * n / tb / 1e9,
                 "fwd_frac_hbm": BYTES_FWD * n / tf / 1e9 / hbm, "bwd_frac_hbm": BYTES_BWD * n / tb / 1e9 / hbm,
                 "fwd_bwd_frac_hbm": (BYTES_FWD + BYTES_BWD) * n / (tf + tb) / 1e9 / hbm,
+                "fwd_refined_matrices_per_s": n / tr, "fwd_refined_frac_hbm": BYTES_FWD * n / tr / 1e9 / hbm,
                 "newton_iters_mean": float(itn.mean()), "newton_iters_max": int(its.max()),
                 "newton_iters_warp_max_mean": float(itn.reshape(-1, 32).max(1).values.mean()),
             })

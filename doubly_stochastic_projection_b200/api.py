@@ -20,7 +20,8 @@ from . import build as _build
 
 SINKHORN = 0
 NEWTON = 1
-_METHODS = {"sinkhorn": SINKHORN, "newton": NEWTON, SINKHORN: SINKHORN, NEWTON: NEWTON}
+NEWTON_REFINED = 2
+_METHODS = {"sinkhorn": SINKHORN, "newton": NEWTON, "newton_refined": NEWTON_REFINED}
 
 _lock = threading.Lock()
 _lib = None
@@ -112,8 +113,9 @@ def birkhoff_fwd(logits: torch.Tensor, method="newton", iters: int = 0, out: tor
     """Project [..., 4, 4] float32 logits onto the Birkhoff polytope.
 
     ``method``: "newton" (exact projection by Newton on the 3-variable reduced
-    dual; ``iters`` = maximum iterations, 0 -> 30) or "sinkhorn" (exactly
-    ``iters`` Sinkhorn-Knopp rounds, 0 -> 20).
+    dual; ``iters`` = maximum iterations, 0 -> 50), "newton_refined" (the same
+    plus a relative-accuracy step for matrices close to a permutation), or
+    "sinkhorn" (exactly ``iters`` Sinkhorn-Knopp rounds, 0 -> 20).
     """
     _need(logits, "logits", torch.float32)
     n = _n_mats(logits)

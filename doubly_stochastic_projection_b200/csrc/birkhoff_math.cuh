@@ -33,6 +33,8 @@ constexpr int kMaxHalvings = 24;
 constexpr float kStepCap = 4.0f;
 // Levenberg-Marquardt damping factor (see newton_project).
 constexpr float kDamping = 0.03f;
+// Largest step (log units) the near-permutation polish may take.
+constexpr float kPolishMaxStep = 0.5f;
 
 // Reciprocal to within 1 ulp (MUFU), flushing subnormals.  Used where a
 // reciprocal only rescales an iterate (normalisations, elimination pivots):
@@ -245,15 +247,30 @@ __device__ __forceinline__ void polish_near_permutation(float (&a)[16])
     const PairWeights w = pair_weights(a);
     float d0, d1, d2;
     if (!laplacian_solve(w, -g[0], -g[1], -g[2], d0, d1, d2)) return;
+    // A converged iterate needs only a small correction.  A long step means
+    // the Laplacian weights (products of entries) have lost their accuracy
+    // to underflow -- entries far below 1e-19 -- and the step is not used.
+    if (!(fmaxf(fmaxf(fabsf(d0), fabsf(d1)), fabsf(d2)) <= kPolishMaxStep)) return;
     const float e0 = __expf(d0), e1 = __expf(d1), e2 = __expf(d2);
+    float b[16];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         const float sr = fmaf(a[4 * r], e0, fmaf(a[4 * r + 1], e1, fmaf(a[4 * r + 2], e2, a[4 * r + 3])));
         const float q = rcp_approx(sr);
-        a[4 * r + 0] *= e0 * q;
-        a[4 * r + 1] *= e1 * q;
-        a[4 * r + 2] *= e2 * q;
-        a[4 * r + 3] *= q;
+        b[4 * r + 0] = a[4 * r + 0] * (e0 * q);
+        b[4 * r + 1] = a[4 * r + 1] * (e1 * q);
+        b[4 * r + 2] = a[4 * r + 2] * (e2 * q);
+        b[4 * r + 3] = a[4 * r + 3] * q;
+    }
+    // keep the polished matrix only if it is still doubly stochastic to the
+    // Newton tolerance
+    float err = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        err = fmaxf(err, fabsf(((b[c] + b[4 + c]) + (b[8 + c] + b[12 + c])) - 1.0f));
+    if (err < kNewtonTol) {
+#pragma unroll
+        for (int k2 = 0; k2 < 16; ++k2) a[k2] = b[k2];
     }
 }
 
@@ -274,10 +291,13 @@ __device__ __forceinline__ void polish_near_permutation(float (&a)[16])
 // proportional to the error, the step capped at kStepCap per potential, and
 // Armijo backtracking on phi while the error is large; a Sinkhorn round
 // replaces the step when the Laplacian is singular or no decrease is found.
-// After convergence, matrices close to a permutation get one more step with
-// a cancellation-free gradient (polish_near_permutation).
+// With kRefine, matrices close to a permutation get one more step after
+// convergence, with a cancellation-free gradient (polish_near_permutation):
+// their small entries become accurate relative to themselves, at the cost of
+// that step (about a third of the time on near-identity inputs).
 // Returns the number of Newton iterations taken (the polish step not counted).
 // ---------------------------------------------------------------------------
+template <bool kRefine = false>
 __device__ __forceinline__ int newton_project(float (&a)[16], int maxit)
 {
     shift_rows_by_max(a);
@@ -367,7 +387,7 @@ __device__ __forceinline__ int newton_project(float (&a)[16], int maxit)
     }
     if (err != err)
         fill_nan(a);  // a non-finite logit poisons its whole matrix
-    else if (err < kNewtonTol)
+    else if (kRefine && err < kNewtonTol)
         polish_near_permutation(a);
     return it;
 }

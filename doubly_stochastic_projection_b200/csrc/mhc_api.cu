@@ -36,7 +36,7 @@ int resolve_iters(int method, int iters, int* out)
     if (iters < 0 || iters > MHC_MAX_ITERS) return MHC_ERR_ARG;
     if (method == MHC_SINKHORN)
         *out = iters == 0 ? mhc::kDefaultSinkhornIters : iters;
-    else if (method == MHC_NEWTON)
+    else if (method == MHC_NEWTON || method == MHC_NEWTON_REFINED)
         *out = iters == 0 ? mhc::kDefaultNewtonIters : iters;
     else
         return MHC_ERR_ARG;
@@ -73,7 +73,8 @@ int mhc_birkhoff_fwd(const float* logits, float* P, int64_t n_mats, int method, 
     if (misaligned(logits) || misaligned(P)) return MHC_ERR_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (method == MHC_SINKHORN) return cuda_status(mhc::launch_sinkhorn_fwd(logits, P, n_mats, it, s));
-    return cuda_status(mhc::launch_newton_fwd(logits, P, nullptr, n_mats, it, s));
+    return cuda_status(
+        mhc::launch_newton_fwd(logits, P, nullptr, n_mats, it, method == MHC_NEWTON_REFINED, s));
 }
 
 int mhc_birkhoff_fwd_diag(const float* logits, float* P, int32_t* iters_out, int64_t n_mats, int iters,
@@ -87,7 +88,7 @@ int mhc_birkhoff_fwd_diag(const float* logits, float* P, int32_t* iters_out, int
     if (!logits || !P || !iters_out) return MHC_ERR_NULL;
     if (misaligned(logits) || misaligned(P) || misaligned(iters_out)) return MHC_ERR_ALIGN;
     return cuda_status(
-        mhc::launch_newton_fwd(logits, P, iters_out, n_mats, it, static_cast<cudaStream_t>(stream)));
+        mhc::launch_newton_fwd(logits, P, iters_out, n_mats, it, false, static_cast<cudaStream_t>(stream)));
 }
 
 int mhc_birkhoff_bwd(const float* logits, const float* P, const float* dP, float* dlogits, int64_t n_mats,

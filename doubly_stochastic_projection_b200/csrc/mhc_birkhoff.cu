@@ -33,7 +33,7 @@ sinkhorn_fwd_kernel(const float* logits, float* P, int64_t n, int iters)
     }
 }
 
-template <bool kDiag>
+template <bool kDiag, bool kRefine>
 __global__ void __launch_bounds__(kProjThreads)
 newton_fwd_kernel(const float* logits, float* P, int32_t* iters_out, int64_t n, int maxit)
 {
@@ -41,7 +41,7 @@ newton_fwd_kernel(const float* logits, float* P, int32_t* iters_out, int64_t n, 
     for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
         float a[16];
         load16(logits + 16 * m, a);
-        const int it = newton_project(a, maxit);
+        const int it = newton_project<kRefine>(a, maxit);
         store16(P + 16 * m, a);
         if (kDiag) iters_out[m] = it;
     }
@@ -105,17 +105,27 @@ cudaError_t launch_sinkhorn_fwd(const float* logits, float* P, int64_t n, int it
     return cudaGetLastError();
 }
 
+template <bool kDiag, bool kRefine>
+static void launch_newton(const float* logits, float* P, int32_t* iters_out, int64_t n, int maxit, cudaStream_t s)
+{
+    const int grid = persistent_grid((const void*)newton_fwd_kernel<kDiag, kRefine>, kProjThreads, 0,
+                                     blocks_for(n, kProjThreads));
+    newton_fwd_kernel<kDiag, kRefine><<<grid, kProjThreads, 0, s>>>(logits, P, iters_out, n, maxit);
+}
+
 cudaError_t launch_newton_fwd(const float* logits, float* P, int32_t* iters_out, int64_t n, int maxit,
-                              cudaStream_t s)
+                              bool refine, cudaStream_t s)
 {
     if (iters_out) {
-        const int grid = persistent_grid((const void*)newton_fwd_kernel<true>, kProjThreads, 0,
-                                         blocks_for(n, kProjThreads));
-        newton_fwd_kernel<true><<<grid, kProjThreads, 0, s>>>(logits, P, iters_out, n, maxit);
+        if (refine)
+            launch_newton<true, true>(logits, P, iters_out, n, maxit, s);
+        else
+            launch_newton<true, false>(logits, P, iters_out, n, maxit, s);
     } else {
-        const int grid = persistent_grid((const void*)newton_fwd_kernel<false>, kProjThreads, 0,
-                                         blocks_for(n, kProjThreads));
-        newton_fwd_kernel<false><<<grid, kProjThreads, 0, s>>>(logits, P, nullptr, n, maxit);
+        if (refine)
+            launch_newton<false, true>(logits, P, nullptr, n, maxit, s);
+        else
+            launch_newton<false, false>(logits, P, nullptr, n, maxit, s);
     }
     return cudaGetLastError();
 }

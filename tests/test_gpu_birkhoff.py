@@ -81,27 +81,48 @@ def test_config2_fwd_bwd_131072(orc):
     assert rel.max() <= GRAD_REL_TOL
 
 
-def test_end_to_end_gradient_against_oracle_projection(orc):
-    # GPU fwd + bwd against the oracle's fwd + bwd on the same logits.  This
-    # includes the fp32 forward's own error, which is absolute (<= 1e-6 on
-    # every entry): on matrices close to a permutation the whole gradient is
-    # proportional to entries of 1e-4 or less, so their per-matrix relative
-    # error is bounded by that absolute error, not by the backward.
-    for dist in ("normal1", "normal3", "normal10", "near_identity", "near_permutation"):
+# End-to-end: GPU fwd + bwd against the oracle's fwd + bwd on the same logits.
+# This includes the fp32 forward's own error.  Plain Newton's P is accurate to
+# ~1e-6 in absolute terms; on matrices close to a permutation the gradient is
+# proportional to entries of 1e-4 or less, so its relative error is bounded by
+# that absolute error (about 1e-3 of those entries), not by the backward.  The
+# refined method makes those entries accurate relative to themselves, and the
+# stricter bar applies to it.
+E2E_BARS = {
+    # method: (median per matrix, p99 per matrix, batch-normalised, per-matrix max where not tiny)
+    "newton_refined": (1e-4, 1e-4, 1e-4, 1e-3),
+    "newton": (1e-4, 1e-3, 5e-4, 5e-3),
+}
+
+
+@pytest.mark.parametrize("method", sorted(E2E_BARS))
+def test_end_to_end_gradient_against_oracle_projection(orc, method):
+    med_bar, p99_bar, batch_bar, big_bar = E2E_BARS[method]
+    for dist in ("normal1", "normal3", "normal10", "near_identity", "near_permutation", "halves_3_deepid"):
         A = inputs.birkhoff_logits(8192, dist, 60)
         G = inputs.upstream_grad(8192, 61)
-        P_g = api.birkhoff_fwd(to_gpu(A), "newton")
+        P_g = api.birkhoff_fwd(to_gpu(A), method)
         dl = to_np64(api.birkhoff_bwd(to_gpu(G), P=P_g))
         ref = orc.implicit_bwd(orc.newton(A.astype(np.float64), tol=1e-13, max_iter=200), G.astype(np.float64))
         rel, scale = per_matrix_rel_err(dl, ref)
-        assert np.median(rel) <= GRAD_REL_TOL, (dist, np.median(rel))
-        # batch-normalised: every entry within 1e-4 of the largest gradient
-        assert np.abs(dl - ref).max() <= GRAD_REL_TOL * np.abs(ref).max(), dist
+        assert np.median(rel) <= med_bar, (dist, np.median(rel))
+        assert np.percentile(rel, 99) <= p99_bar, (dist, np.percentile(rel, 99))
+        assert np.abs(dl - ref).max() <= batch_bar * np.abs(ref).max(), (dist, np.abs(dl - ref).max() / np.abs(ref).max())
         # per matrix, wherever the gradient is not itself at the scale of the
-        # forward's absolute error
-        big = scale >= 1e-2 * np.abs(G).reshape(-1, 16).max(1)
-        assert big.mean() > 0.5
-        assert rel[big].max() <= 1e-3, (dist, rel[big].max())
+        # forward's absolute error (entries of P below ~1e-6)
+        big = scale >= 1e-4 * np.abs(G).reshape(-1, 16).max(1)
+        assert rel[big].max() <= big_bar, (dist, rel[big].max())
+
+
+def test_refined_forward_parity(orc):
+    for dist in ("normal1", "normal10", "near_identity", "near_permutation"):
+        A = inputs.birkhoff_logits(20000, dist, 62)
+        P = _newton_checks(api.birkhoff_fwd(to_gpu(A), "newton_refined"), A, orc)
+        ref = orc.newton(A.astype(np.float64), tol=1e-13, max_iter=200)
+        # entries of the refined projection are accurate relative to themselves
+        if dist in ("near_identity", "near_permutation"):
+            small = ref < 0.5
+            assert (np.abs(P - ref)[small] <= 1e-5 * ref[small] + 1e-12).all()
 
 
 @pytest.mark.parametrize("si", range(len(inputs.SWEEP_SIZES)))
