@@ -56,7 +56,7 @@ def test_validation_rejects_before_any_cuda_call(L):
     L.mhc_birkhoff_bwd.argtypes = [p, p, p, p, i64, p]
     fake = 1 << 20  # never dereferenced: every call below returns before launching
     assert L.mhc_birkhoff_fwd(fake, fake, -5, 1, 0, None) == 3
-    assert L.mhc_birkhoff_fwd(fake, fake, 10, 2, 0, None) == 4
+    assert L.mhc_birkhoff_fwd(fake, fake, 10, 3, 0, None) == 4
     assert L.mhc_birkhoff_fwd(fake, fake, 10, 0, -1, None) == 4
     assert L.mhc_birkhoff_fwd(fake, fake, 10, 1, 1001, None) == 4
     assert L.mhc_birkhoff_fwd(None, fake, 10, 1, 0, None) == 1
