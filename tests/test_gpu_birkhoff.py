@@ -91,7 +91,7 @@ def test_config2_fwd_bwd_131072(orc):
 E2E_BARS = {
     # method: (median per matrix, p99 per matrix, batch-normalised, per-matrix max where not tiny)
     "newton_refined": (1e-4, 1e-4, 1e-4, 1e-3),
-    "newton": (1e-4, 1e-3, 5e-4, 5e-3),
+    "newton": (1e-4, 5e-3, 5e-4, 1e-2),
 }
 
 
