@@ -20,6 +20,12 @@ namespace mhc {
 namespace {
 
 constexpr int kProjThreads = 256;
+// Batches that fit in about two waves of 256-thread CTAs are launched with
+// 128-thread CTAs instead: twice as many CTAs spread the batch (and its mix
+// of easy and hard matrices) more evenly over the 148 SMs.  Measured on B200:
+// 131072 matrices, Newton 18.4 -> 16.4 us, backward 12.3 -> 11.2 us; at 16M
+// matrices 256-thread CTAs are 1-2% faster.
+constexpr int kProjThreadsSmall = 128;
 
 __global__ void __launch_bounds__(kProjThreads)
 sinkhorn_fwd_kernel(const float* logits, float* P, int64_t n, int iters)
@@ -70,6 +76,21 @@ implicit_bwd_kernel(const float* logits, const float* P, const float* dP, float*
 
 int64_t blocks_for(int64_t n, int threads) { return (n + threads - 1) / threads; }
 
+// Threads per CTA and grid size for a grid-stride projection kernel.
+struct Launch {
+    int threads, grid;
+};
+
+Launch projection_launch(const void* kernel, int64_t n)
+{
+    const int full = persistent_grid(kernel, kProjThreads, 0, int64_t(1) << 40);
+    if (blocks_for(n, kProjThreads) <= 2 * (int64_t)full) {
+        const int g = persistent_grid(kernel, kProjThreadsSmall, 0, blocks_for(n, kProjThreadsSmall));
+        return {kProjThreadsSmall, g};
+    }
+    return {kProjThreads, full};
+}
+
 }  // namespace
 
 int device_sm_count()
@@ -99,18 +120,16 @@ int persistent_grid(const void* kernel, int threads, size_t smem, int64_t blocks
 
 cudaError_t launch_sinkhorn_fwd(const float* logits, float* P, int64_t n, int iters, cudaStream_t s)
 {
-    const void* k = (const void*)sinkhorn_fwd_kernel;
-    const int grid = persistent_grid(k, kProjThreads, 0, blocks_for(n, kProjThreads));
-    sinkhorn_fwd_kernel<<<grid, kProjThreads, 0, s>>>(logits, P, n, iters);
+    const Launch L = projection_launch((const void*)sinkhorn_fwd_kernel, n);
+    sinkhorn_fwd_kernel<<<L.grid, L.threads, 0, s>>>(logits, P, n, iters);
     return cudaGetLastError();
 }
 
 template <bool kDiag, bool kRefine>
 static void launch_newton(const float* logits, float* P, int32_t* iters_out, int64_t n, int maxit, cudaStream_t s)
 {
-    const int grid = persistent_grid((const void*)newton_fwd_kernel<kDiag, kRefine>, kProjThreads, 0,
-                                     blocks_for(n, kProjThreads));
-    newton_fwd_kernel<kDiag, kRefine><<<grid, kProjThreads, 0, s>>>(logits, P, iters_out, n, maxit);
+    const Launch L = projection_launch((const void*)newton_fwd_kernel<kDiag, kRefine>, n);
+    newton_fwd_kernel<kDiag, kRefine><<<L.grid, L.threads, 0, s>>>(logits, P, iters_out, n, maxit);
 }
 
 cudaError_t launch_newton_fwd(const float* logits, float* P, int32_t* iters_out, int64_t n, int maxit,
@@ -134,13 +153,11 @@ cudaError_t launch_implicit_bwd(const float* logits, const float* P, const float
                                 int64_t n, cudaStream_t s)
 {
     if (P) {
-        const int grid = persistent_grid((const void*)implicit_bwd_kernel<false>, kProjThreads, 0,
-                                         blocks_for(n, kProjThreads));
-        implicit_bwd_kernel<false><<<grid, kProjThreads, 0, s>>>(nullptr, P, dP, dlogits, n);
+        const Launch L = projection_launch((const void*)implicit_bwd_kernel<false>, n);
+        implicit_bwd_kernel<false><<<L.grid, L.threads, 0, s>>>(nullptr, P, dP, dlogits, n);
     } else {
-        const int grid = persistent_grid((const void*)implicit_bwd_kernel<true>, kProjThreads, 0,
-                                         blocks_for(n, kProjThreads));
-        implicit_bwd_kernel<true><<<grid, kProjThreads, 0, s>>>(logits, nullptr, dP, dlogits, n);
+        const Launch L = projection_launch((const void*)implicit_bwd_kernel<true>, n);
+        implicit_bwd_kernel<true><<<L.grid, L.threads, 0, s>>>(logits, nullptr, dP, dlogits, n);
     }
     return cudaGetLastError();
 }
