@@ -44,13 +44,14 @@ def _load():
             lib = ctypes.CDLL(build())
             i64, i32, dbl, p = ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_void_p
             lib.oracle_sinkhorn.argtypes = [p, p, i64, i32, i32]
+            lib.oracle_sinkhorn_bwd.argtypes = [p, p, p, i64, i32, i32]
             lib.oracle_newton.argtypes = [p, p, i64, i32, dbl, i32, p, p]
             lib.oracle_implicit_bwd.argtypes = [p, p, p, i64, i32]
             lib.oracle_mix_fwd.argtypes = [p, p, p, p, p, i64, i32, i64]
             lib.oracle_mix_bwd.argtypes = [p, p, p, p, p, p, p, p, p, i64, i32, i64]
             lib.oracle_set_threads.argtypes = [i32]
             lib.oracle_get_threads.restype = i32
-            for f in (lib.oracle_sinkhorn, lib.oracle_newton, lib.oracle_implicit_bwd,
+            for f in (lib.oracle_sinkhorn, lib.oracle_sinkhorn_bwd, lib.oracle_newton, lib.oracle_implicit_bwd,
                       lib.oracle_mix_fwd, lib.oracle_mix_bwd):
                 f.restype = i32
             _lib = lib
@@ -104,6 +105,24 @@ def sinkhorn(A, iters: int = 20) -> np.ndarray:
     if rc != 0:
         raise ValueError("oracle_sinkhorn: bad arguments")
     return P
+
+
+def sinkhorn_bwd(A, G, iters: int = 20) -> np.ndarray:
+    """dL/dA through the fixed-count Sinkhorn-Knopp forward, by reverse-mode
+    differentiation of the unrolled iteration (iterates stored, fp64).
+
+    Birkhoff-acceleration summary (arXiv 2606.07574) §1: the backward of the
+    Sinkhorn baseline unrolls the iteration.
+    """
+    A = _mats(A)
+    G = _mats(G)
+    if A.shape != G.shape:
+        raise ValueError("A and G shapes differ")
+    dA = np.empty_like(A)
+    rc = _load().oracle_sinkhorn_bwd(_ptr(A), _ptr(G), _ptr(dA), A.shape[0], A.shape[1], int(iters))
+    if rc != 0:
+        raise ValueError("oracle_sinkhorn_bwd: bad arguments")
+    return dA
 
 
 def newton(A, tol: float = 1e-10, max_iter: int = 100, return_info: bool = False):

@@ -192,6 +192,85 @@ int oracle_sinkhorn(const double *A, double *P, int64_t n_mats, int n, int iters
     return 0;
 }
 
+/* Vector-Jacobian product of the fixed-count Sinkhorn-Knopp forward
+ * (sinkhorn_one above), by plain reverse-mode differentiation: every
+ * half-step's input is stored on the forward pass, then the chain rule is
+ * applied backwards.  For a normalisation Y = X / s (s the row or column
+ * sums of X) the derivative is dX = (dY - sum(dY * Y)) / s along that row
+ * or column.  The row max shift cancels in the first row normalisation and
+ * contributes nothing.  This is what an autograd framework computes when it
+ * unrolls the iteration ([BA] §1 names that unrolled backward as the
+ * baseline the implicit method replaces). */
+static void sinkhorn_vjp_one(int n, const double *A, const double *G, double *dA, int iters)
+{
+    const int nn = n * n;
+    double *X = (double *)malloc(sizeof(double) * (size_t)nn * (size_t)(2 * iters + 1));
+    double *g = (double *)malloc(sizeof(double) * (size_t)nn);
+    double *h = (double *)malloc(sizeof(double) * (size_t)nn);
+    /* X[0] = exp(A - rowmax); X[2t+1] = rows of X[2t] normalised;
+     * X[2t+2] = columns of X[2t+1] normalised */
+    for (int i = 0; i < n; ++i) {
+        double m = A[i * n];
+        for (int j = 1; j < n; ++j)
+            if (A[i * n + j] > m) m = A[i * n + j];
+        for (int j = 0; j < n; ++j) X[i * n + j] = exp(A[i * n + j] - m);
+    }
+    for (int t = 0; t < iters; ++t) {
+        const double *in = X + (size_t)(2 * t) * nn;
+        double *y = X + (size_t)(2 * t + 1) * nn;
+        double *z = X + (size_t)(2 * t + 2) * nn;
+        for (int i = 0; i < n; ++i) {
+            double s = 0.0;
+            for (int j = 0; j < n; ++j) s += in[i * n + j];
+            for (int j = 0; j < n; ++j) y[i * n + j] = in[i * n + j] / s;
+        }
+        for (int j = 0; j < n; ++j) {
+            double s = 0.0;
+            for (int i = 0; i < n; ++i) s += y[i * n + j];
+            for (int i = 0; i < n; ++i) z[i * n + j] = y[i * n + j] / s;
+        }
+    }
+    for (int q = 0; q < nn; ++q) g[q] = G[q];
+    for (int t = iters - 1; t >= 0; --t) {
+        const double *in = X + (size_t)(2 * t) * nn;
+        const double *y = X + (size_t)(2 * t + 1) * nn;
+        const double *z = X + (size_t)(2 * t + 2) * nn;
+        /* through the column normalisation z = y / colsum(y) */
+        for (int j = 0; j < n; ++j) {
+            double s = 0.0, dot = 0.0;
+            for (int i = 0; i < n; ++i) {
+                s += y[i * n + j];
+                dot += g[i * n + j] * z[i * n + j];
+            }
+            for (int i = 0; i < n; ++i) h[i * n + j] = (g[i * n + j] - dot) / s;
+        }
+        /* through the row normalisation y = in / rowsum(in) */
+        for (int i = 0; i < n; ++i) {
+            double s = 0.0, dot = 0.0;
+            for (int j = 0; j < n; ++j) {
+                s += in[i * n + j];
+                dot += h[i * n + j] * y[i * n + j];
+            }
+            for (int j = 0; j < n; ++j) g[i * n + j] = (h[i * n + j] - dot) / s;
+        }
+    }
+    /* through K = exp(A - rowmax A) */
+    for (int q = 0; q < nn; ++q) dA[q] = g[q] * X[q];
+    free(X);
+    free(g);
+    free(h);
+}
+
+int oracle_sinkhorn_bwd(const double *A, const double *G, double *dA, int64_t n_mats, int n, int iters)
+{
+    if (n < 1 || n > ORACLE_NMAX || n_mats < 0 || iters < 1) return -1;
+    const int64_t nn = (int64_t)n * n;
+#pragma omp parallel for schedule(dynamic, 256)
+    for (int64_t m = 0; m < n_mats; ++m)
+        sinkhorn_vjp_one(n, A + m * nn, G + m * nn, dA + m * nn, iters);
+    return 0;
+}
+
 /* ------------------------------------------------------------------ */
 /* Newton's method on the reduced entropic-OT dual                    */
 /* ------------------------------------------------------------------ */

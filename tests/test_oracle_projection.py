@@ -262,3 +262,43 @@ def test_implicit_bwd_invariances(orc):
     assert np.abs(orc.implicit_bwd(P, G + a + b) - dA).max() < 1e-12
     # n = 1: the projection is constant
     assert np.array_equal(orc.implicit_bwd(np.ones((2, 1, 1)), np.ones((2, 1, 1))), np.zeros((2, 1, 1)))
+
+
+# ---------------------------------------------------------------- Sinkhorn backward
+
+
+@pytest.mark.parametrize("iters", [1, 3, 20])
+def test_sinkhorn_bwd_matches_finite_differences(orc, iters):
+    rng = np.random.default_rng(30 + iters)
+    for n, scale in ((2, 1.0), (4, 1.0), (4, 4.0), (5, 2.0)):
+        A = rng.standard_normal((300, n, n)) * scale
+        G = rng.standard_normal((300, n, n))
+        dA = orc.sinkhorn_bwd(A, G, iters)
+        fd = np.zeros_like(A)
+        h = 1e-6
+        for i in range(n):
+            for j in range(n):
+                Ap = A.copy()
+                Ap[:, i, j] += h
+                Am = A.copy()
+                Am[:, i, j] -= h
+                fd[:, i, j] = ((orc.sinkhorn(Ap, iters) - orc.sinkhorn(Am, iters)) * G).sum((1, 2)) / (2 * h)
+        assert np.abs(dA - fd).max() <= 1e-7 * max(1.0, np.abs(fd).max()), (n, iters)
+
+
+def test_sinkhorn_bwd_invariances(orc):
+    A = _logits("normal3", n=200, seed=33)
+    rng = np.random.default_rng(34)
+    G = rng.standard_normal((200, 4, 4))
+    dA = orc.sinkhorn_bwd(A, G, 20)
+    # row shifts of A cancel in the first row normalisation: zero row sums
+    assert np.abs(dA.sum(2)).max() < 1e-12
+    # the last half-step normalises columns: an upstream 1 b^T is orthogonal
+    b = rng.standard_normal((200, 1, 4))
+    assert np.abs(orc.sinkhorn_bwd(A, G + b, 20) - dA).max() < 1e-12
+    # converged Sinkhorn approaches the implicit (Newton) gradient
+    A1 = _logits("normal1", n=100, seed=35)
+    G1 = rng.standard_normal((100, 4, 4))
+    d_sk = orc.sinkhorn_bwd(A1, G1, 3000)
+    d_nt = orc.implicit_bwd(orc.newton(A1, tol=1e-14), G1)
+    assert np.abs(d_sk - d_nt).max() < 1e-8
