@@ -345,6 +345,25 @@ def extras(dev, stream, flush, hbm, api, inputs):
                                           "fwd_frac_hbm": BYTES_FWD * n / ts / 1e9 / hbm})
             del A, G, P, dl, its
             torch.cuda.empty_cache()
+    # The pages' comparison (Birkhoff-acceleration summary, section 4): forward +
+    # backward of the Newton projection with the implicit backward, against
+    # 20-round Sinkhorn with the backward through the unrolled iteration.
+    out["newton_vs_sinkhorn20_fwd_bwd"] = []
+    for n, dist, seed in ((131072, "halves_1_10", 2), (1 << 20, "normal1", 300), (1 << 24, "normal1", 320),
+                          (1 << 24, "normal10", 322)):
+        A = torch.from_numpy(inputs.birkhoff_logits(n, dist, seed)).to(dev)
+        G = torch.from_numpy(inputs.upstream_grad(n, seed + 1000)).to(dev)
+        P = torch.empty_like(A)
+        dl = torch.empty_like(A)
+        t_nt = event_time(lambda: (api.birkhoff_fwd(A, "newton", out=P), api.birkhoff_bwd(G, P=P, out=dl)),
+                          reps, stream, flush)
+        t_sk = event_time(lambda: (api.birkhoff_fwd(A, "sinkhorn", 20, out=P), api.sinkhorn_bwd(G, A, 20, out=dl)),
+                          reps, stream, flush)
+        out["newton_vs_sinkhorn20_fwd_bwd"].append({
+            "n_mats": n, "dist": dist, "newton_implicit_matrices_per_s": n / t_nt,
+            "sinkhorn20_unrolled_matrices_per_s": n / t_sk, "speedup": t_sk / t_nt})
+        del A, G, P, dl
+        torch.cuda.empty_cache()
     for name in ("mix_T16384_C4096", "mix_T65536_C7168"):
         m = inputs.mix_workload(name, device=dev)
         T, C = m["T"], m["C"]

@@ -55,6 +55,7 @@ def lib() -> ctypes.CDLL:
                 "mhc_birkhoff_fwd": [p, p, i64, i32, i32, p],
                 "mhc_birkhoff_fwd_diag": [p, p, p, i64, i32, p],
                 "mhc_birkhoff_bwd": [p, p, p, p, i64, p],
+                "mhc_sinkhorn_bwd": [p, p, p, i64, i32, p],
                 "mhc_residual_mix_fwd": [p, p, p, p, p, i64, i64, p],
                 "mhc_residual_mix_bwd": [p, p, p, p, p, p, p, p, p, p, i64, i64, p],
                 "mhc_proj_mix_fwd": [p, p, p, p, p, p, i64, i64, i32, p],
@@ -151,6 +152,19 @@ def birkhoff_bwd(dP: torch.Tensor, P: torch.Tensor | None = None, logits: torch.
         out = torch.empty_like(dP)
     _need(out, "out", torch.float32, dP.shape)
     _check(lib().mhc_birkhoff_bwd(_ptr(logits), _ptr(P), _ptr(dP), _ptr(out), n, _stream(dP)))
+    return out
+
+
+def sinkhorn_bwd(dP: torch.Tensor, logits: torch.Tensor, iters: int = 20, out: torch.Tensor | None = None):
+    """Backward of the fixed-count Sinkhorn forward (same ``iters``): dlogits from
+    the upstream dP and the forward's logits, iterates recomputed in-kernel."""
+    _need(dP, "dP", torch.float32)
+    n = _n_mats(dP)
+    _need(logits, "logits", torch.float32, dP.shape)
+    if out is None:
+        out = torch.empty_like(dP)
+    _need(out, "out", torch.float32, dP.shape)
+    _check(lib().mhc_sinkhorn_bwd(_ptr(logits), _ptr(dP), _ptr(out), n, int(iters), _stream(dP)))
     return out
 
 

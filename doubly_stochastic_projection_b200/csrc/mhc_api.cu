@@ -103,6 +103,18 @@ int mhc_birkhoff_bwd(const float* logits, const float* P, const float* dP, float
         mhc::launch_implicit_bwd(logits, P, dP, dlogits, n_mats, static_cast<cudaStream_t>(stream)));
 }
 
+int mhc_sinkhorn_bwd(const float* logits, const float* dP, float* dlogits, int64_t n_mats, int iters, void* stream)
+{
+    int rc = check_matrices(n_mats);
+    if (rc != MHC_OK) return rc;
+    int it = 0;
+    if ((rc = resolve_iters(MHC_SINKHORN, iters, &it)) != MHC_OK) return rc;
+    if (n_mats == 0) return MHC_OK;
+    if (!logits || !dP || !dlogits) return MHC_ERR_NULL;
+    if (misaligned(logits) || misaligned(dP) || misaligned(dlogits)) return MHC_ERR_ALIGN;
+    return cuda_status(mhc::launch_sinkhorn_bwd(logits, dP, dlogits, n_mats, it, static_cast<cudaStream_t>(stream)));
+}
+
 int mhc_residual_mix_fwd(const uint16_t* X, const float* H_res, const float* h_post, const uint16_t* F,
                          uint16_t* Y, int64_t T, int64_t C, void* stream)
 {

@@ -74,6 +74,19 @@ implicit_bwd_kernel(const float* logits, const float* P, const float* dP, float*
     }
 }
 
+__global__ void __launch_bounds__(kProjThreads)
+sinkhorn_bwd_kernel(const float* logits, const float* dP, float* dlogits, int64_t n, int iters)
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
+        float a[16], g[16], out[16];
+        load16(logits + 16 * m, a);
+        load16(dP + 16 * m, g);
+        sinkhorn_vjp(a, g, iters, out);
+        store16(dlogits + 16 * m, out);
+    }
+}
+
 int64_t blocks_for(int64_t n, int threads) { return (n + threads - 1) / threads; }
 
 // Threads per CTA and grid size for a grid-stride projection kernel.
@@ -159,6 +172,14 @@ cudaError_t launch_implicit_bwd(const float* logits, const float* P, const float
         const Launch L = projection_launch((const void*)implicit_bwd_kernel<true>, n);
         implicit_bwd_kernel<true><<<L.grid, L.threads, 0, s>>>(logits, nullptr, dP, dlogits, n);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_sinkhorn_bwd(const float* logits, const float* dP, float* dlogits, int64_t n, int iters,
+                                cudaStream_t s)
+{
+    const Launch L = projection_launch((const void*)sinkhorn_bwd_kernel, n);
+    sinkhorn_bwd_kernel<<<L.grid, L.threads, 0, s>>>(logits, dP, dlogits, n, iters);
     return cudaGetLastError();
 }
 

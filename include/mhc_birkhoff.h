@@ -153,6 +153,21 @@ MHC_API int mhc_birkhoff_bwd(const float *logits, const float *P, const float *d
                      int64_t n_mats, void *stream);
 
 /*
+ * mhc_sinkhorn_bwd -- backward of the MHC_SINKHORN forward with the same
+ * `iters`: dlogits = dL/dlogits for upstream dP = dL/dP, the exact derivative
+ * of the fixed-count iteration (the unrolled backward of the Sinkhorn baseline
+ * the implicit method replaces, [BA] §1).  Nothing is saved by the forward:
+ * the iterates are recomputed in registers, segment by segment.
+ *
+ *   logits  [n_mats][4][4] float, read (the forward's input).
+ *   dP      [n_mats][4][4] float, read.
+ *   dlogits [n_mats][4][4] float, written.  May alias dP.
+ *   iters   1 .. MHC_MAX_ITERS, or 0 for 20 (must match the forward).
+ */
+MHC_API int mhc_sinkhorn_bwd(const float *logits, const float *dP, float *dlogits, int64_t n_mats,
+                             int iters, void *stream);
+
+/*
  * mhc_residual_mix_fwd -- Y = H_res . X + h_post (x) F per token:
  *     Y[t,i,c] = sum_j H_res[t,i,j] X[t,j,c] + h_post[t,i] F[t,c]
  * The widened residual of n = 4 parallel streams is mixed by the per-token

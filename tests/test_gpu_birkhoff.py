@@ -210,3 +210,30 @@ def test_argument_errors():
     with pytest.raises(ValueError):
         api.birkhoff_fwd(A.cpu())
     torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------ Sinkhorn backward
+
+
+@pytest.mark.parametrize("iters", [1, 5, 20])
+def test_sinkhorn_bwd_parity(orc, iters):
+    for dist in ("normal1", "normal10", "near_permutation"):
+        n = 4096 + 37
+        A = inputs.birkhoff_logits(n, dist, 80)
+        G = inputs.upstream_grad(n, 81)
+        dl = to_np64(api.sinkhorn_bwd(to_gpu(G), to_gpu(A), iters))
+        ref = orc.sinkhorn_bwd(A.astype(np.float64), G.astype(np.float64), iters)
+        rel, _ = per_matrix_rel_err(dl, ref)
+        assert np.median(rel) <= GRAD_REL_TOL, (dist, iters, np.median(rel))
+        assert np.abs(dl - ref).max() <= GRAD_REL_TOL * np.abs(ref).max(), (dist, iters)
+        # row shifts cancel in the first row normalisation
+        assert np.abs(dl.sum(-1)).max() <= 1e-5 * np.abs(dl).max()
+
+
+def test_sinkhorn_fwd_bwd_config2(orc):
+    A, G = inputs.birkhoff_workload("birkhoff_fwd_bwd_131072")
+    dl = to_np64(api.sinkhorn_bwd(to_gpu(G), to_gpu(A), 20))
+    ref = orc.sinkhorn_bwd(A.astype(np.float64), G.astype(np.float64), 20)
+    rel, _ = per_matrix_rel_err(dl, ref)
+    assert np.median(rel) <= GRAD_REL_TOL
+    assert np.abs(dl - ref).max() <= GRAD_REL_TOL * np.abs(ref).max()
