@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
                 "mhc_birkhoff_fwd_diag": [p, p, p, i64, i32, p],
                 "mhc_birkhoff_bwd": [p, p, p, p, i64, p],
                 "mhc_sinkhorn_bwd": [p, p, p, i64, i32, p],
+                "mhc_birkhoff_fwd_n": [p, p, i64, i32, i32, i32, p],
+                "mhc_birkhoff_bwd_n": [p, p, p, i64, i32, p],
                 "mhc_residual_mix_fwd": [p, p, p, p, p, i64, i64, p],
                 "mhc_residual_mix_bwd": [p, p, p, p, p, p, p, p, p, p, i64, i64, p],
                 "mhc_proj_mix_fwd": [p, p, p, p, p, p, i64, i64, i32, p],
@@ -152,6 +154,37 @@ def birkhoff_bwd(dP: torch.Tensor, P: torch.Tensor | None = None, logits: torch.
         out = torch.empty_like(dP)
     _need(out, "out", torch.float32, dP.shape)
     _check(lib().mhc_birkhoff_bwd(_ptr(logits), _ptr(P), _ptr(dP), _ptr(out), n, _stream(dP)))
+    return out
+
+
+def _square(t, name):
+    if t.dim() < 2 or t.shape[-1] != t.shape[-2]:
+        raise ValueError("%s must be [..., n, n], got %s" % (name, tuple(t.shape)))
+    n = int(t.shape[-1])
+    return n, (t.numel() // (n * n) if n else 0)
+
+
+def birkhoff_fwd_n(logits: torch.Tensor, method="newton", iters: int = 0, out: torch.Tensor | None = None):
+    """Projection of [..., n, n] float32 logits, n = 1..8 (see birkhoff_fwd)."""
+    _need(logits, "logits", torch.float32)
+    n, count = _square(logits, "logits")
+    if out is None:
+        out = torch.empty_like(logits)
+    _need(out, "out", torch.float32, logits.shape)
+    m = _METHODS.get(method, -1) if not isinstance(method, int) else method
+    _check(lib().mhc_birkhoff_fwd_n(_ptr(logits), _ptr(out), count, n, int(m), int(iters), _stream(logits)))
+    return out
+
+
+def birkhoff_bwd_n(dP: torch.Tensor, P: torch.Tensor, out: torch.Tensor | None = None):
+    """Implicit backward for [..., n, n] projections, n = 1..8."""
+    _need(dP, "dP", torch.float32)
+    n, count = _square(dP, "dP")
+    _need(P, "P", torch.float32, dP.shape)
+    if out is None:
+        out = torch.empty_like(dP)
+    _need(out, "out", torch.float32, dP.shape)
+    _check(lib().mhc_birkhoff_bwd_n(_ptr(P), _ptr(dP), _ptr(out), count, n, _stream(dP)))
     return out
 
 

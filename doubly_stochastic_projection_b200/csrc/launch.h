@@ -23,6 +23,12 @@ cudaError_t launch_sinkhorn_bwd(const float* logits, const float* dP, float* dlo
 cudaError_t launch_implicit_bwd(const float* logits, const float* P, const float* dP, float* dlogits,
                                 int64_t n, cudaStream_t s);
 
+// n x n projection, n = 1..8 (n = 4 goes to the 4 x 4 kernels above).
+cudaError_t launch_birkhoff_fwd_n(const float* logits, float* P, int64_t n_mats, int n, bool newton, int iters,
+                                  cudaStream_t s);
+cudaError_t launch_implicit_bwd_n(const float* P, const float* dP, float* dlogits, int64_t n_mats, int n,
+                                  cudaStream_t s);
+
 cudaError_t launch_mix_fwd(const uint16_t* X, const float* H, const float* hpost, const uint16_t* F,
                            uint16_t* Y, int64_t T, int64_t C, cudaStream_t s);
 cudaError_t launch_mix_bwd(const uint16_t* X, const float* H, const float* hpost, const uint16_t* F,

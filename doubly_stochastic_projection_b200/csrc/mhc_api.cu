@@ -103,6 +103,34 @@ int mhc_birkhoff_bwd(const float* logits, const float* P, const float* dP, float
         mhc::launch_implicit_bwd(logits, P, dP, dlogits, n_mats, static_cast<cudaStream_t>(stream)));
 }
 
+int mhc_birkhoff_fwd_n(const float* logits, float* P, int64_t n_mats, int n, int method, int iters, void* stream)
+{
+    if (n < 1 || n > 8) return MHC_ERR_SIZE;
+    int rc = check_matrices(n_mats);
+    if (rc != MHC_OK) return rc;
+    if (method == MHC_NEWTON_REFINED && n != 4) return MHC_ERR_ARG;
+    int it = 0;
+    if ((rc = resolve_iters(method, iters, &it)) != MHC_OK) return rc;
+    if (n_mats == 0) return MHC_OK;
+    if (!logits || !P) return MHC_ERR_NULL;
+    if (misaligned(logits) || misaligned(P)) return MHC_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (n == 4 && method == MHC_NEWTON_REFINED)
+        return cuda_status(mhc::launch_newton_fwd(logits, P, nullptr, n_mats, it, true, s));
+    return cuda_status(mhc::launch_birkhoff_fwd_n(logits, P, n_mats, n, method != MHC_SINKHORN, it, s));
+}
+
+int mhc_birkhoff_bwd_n(const float* P, const float* dP, float* dlogits, int64_t n_mats, int n, void* stream)
+{
+    if (n < 1 || n > 8) return MHC_ERR_SIZE;
+    int rc = check_matrices(n_mats);
+    if (rc != MHC_OK) return rc;
+    if (n_mats == 0) return MHC_OK;
+    if (!P || !dP || !dlogits) return MHC_ERR_NULL;
+    if (misaligned(P) || misaligned(dP) || misaligned(dlogits)) return MHC_ERR_ALIGN;
+    return cuda_status(mhc::launch_implicit_bwd_n(P, dP, dlogits, n_mats, n, static_cast<cudaStream_t>(stream)));
+}
+
 int mhc_sinkhorn_bwd(const float* logits, const float* dP, float* dlogits, int64_t n_mats, int iters, void* stream)
 {
     int rc = check_matrices(n_mats);

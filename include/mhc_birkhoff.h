@@ -153,6 +153,24 @@ MHC_API int mhc_birkhoff_bwd(const float *logits, const float *P, const float *d
                      int64_t n_mats, void *stream);
 
 /*
+ * mhc_birkhoff_fwd_n / mhc_birkhoff_bwd_n -- the projection and its implicit
+ * backward for n x n matrices, n = 1..8: other expansion rates of the
+ * residual stream (the dual then has n - 1 free variables, [BA] §2.1; n = 1
+ * reduces to the scalar 1, [NA]).  Same methods, tolerances and conventions
+ * as mhc_birkhoff_fwd / mhc_birkhoff_bwd; MHC_NEWTON_REFINED is accepted for
+ * n = 4 only.  n = 4 runs the 4 x 4 kernels.
+ *
+ *   logits, P, dP, dlogits  [n_mats][n][n] float, device, row-major.
+ *   n  1..8 (MHC_ERR_SIZE otherwise).
+ *   The base pointers must be 16-byte aligned like every other argument; the
+ *   matrices themselves are read element by element.
+ */
+MHC_API int mhc_birkhoff_fwd_n(const float *logits, float *P, int64_t n_mats, int n, int method,
+                               int iters, void *stream);
+MHC_API int mhc_birkhoff_bwd_n(const float *P, const float *dP, float *dlogits, int64_t n_mats, int n,
+                               void *stream);
+
+/*
  * mhc_sinkhorn_bwd -- backward of the MHC_SINKHORN forward with the same
  * `iters`: dlogits = dL/dlogits for upstream dP = dL/dP, the exact derivative
  * of the fixed-count iteration (the unrolled backward of the Sinkhorn baseline

@@ -67,3 +67,7 @@ def test_validation_rejects_before_any_cuda_call(L):
     assert L.mhc_residual_mix_fwd(fake, fake, fake, fake, fake, 4, 0, None) == 3
     assert L.mhc_residual_mix_fwd(fake, fake, fake, fake, fake + 8, 4, 16, None) == 2
     assert L.mhc_residual_mix_fwd(None, None, None, None, None, 0, 16, None) == 0
+    L.mhc_birkhoff_fwd_n.argtypes = [p, p, i64, i32, i32, i32, p]
+    assert L.mhc_birkhoff_fwd_n(fake, fake, 10, 9, 1, 0, None) == 3
+    assert L.mhc_birkhoff_fwd_n(fake, fake, 10, 5, 2, 0, None) == 4
+    assert L.mhc_birkhoff_fwd_n(None, None, 0, 5, 1, 0, None) == 0

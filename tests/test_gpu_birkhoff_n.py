@@ -1,0 +1,64 @@
+"""GPU parity of the n x n projection (n = 1..8, other expansion rates) against
+the fp64 oracle, which is generic in n, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+from doubly_stochastic_projection_b200 import api
+from _gpu_util import GRAD_REL_TOL, P_ABS_TOL, SUM_TOL, dev, per_matrix_rel_err, row_normalised, to_gpu, to_np64
+
+pytestmark = pytest.mark.gpu
+
+
+def _logits(count, n, sigma, seed):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((count, n, n)) * sigma).astype(np.float32)
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 5, 6, 7, 8])
+@pytest.mark.parametrize("sigma", [1.0, 3.0])
+def test_projection_n_parity(orc, n, sigma):
+    count = 2048 + 13
+    A = _logits(count, n, sigma, 100 + n)
+    G = _logits(count, n, 1.0, 200 + n)
+    P_g = api.birkhoff_fwd_n(to_gpu(A), "newton")
+    P = to_np64(P_g)
+    ref = orc.newton(A.astype(np.float64), tol=1e-12, max_iter=200)
+    assert np.isfinite(P).all() and P.min() >= 0
+    assert np.abs(P.sum(-1) - 1).max() <= SUM_TOL and np.abs(P.sum(-2) - 1).max() <= SUM_TOL
+    assert np.abs(P - ref).max() <= P_ABS_TOL
+    S = to_np64(api.birkhoff_fwd_n(to_gpu(A), "sinkhorn", 20))
+    assert np.abs(S - orc.sinkhorn(A.astype(np.float64), 20)).max() <= P_ABS_TOL
+    dl = to_np64(api.birkhoff_bwd_n(to_gpu(G), P_g))
+    dref = orc.implicit_bwd(row_normalised(P), G.astype(np.float64))
+    if n == 1:
+        assert np.array_equal(dl, np.zeros_like(dl))
+    else:
+        rel, _ = per_matrix_rel_err(dl.reshape(count, -1), dref.reshape(count, -1))
+        assert rel.max() <= GRAD_REL_TOL, (n, sigma, rel.max())
+
+
+def test_n2_closed_form():
+    A = _logits(5000, 2, 4.0, 7)
+    P = to_np64(api.birkhoff_fwd_n(to_gpu(A), "newton"))
+    d = A[:, 0, 0].astype(np.float64) + A[:, 1, 1] - A[:, 0, 1] - A[:, 1, 0]
+    p = 1.0 / (1.0 + np.exp(-d / 2))
+    assert np.abs(P[:, 0, 0] - p).max() <= 2e-6 and np.abs(P[:, 0, 1] - (1 - p)).max() <= 2e-6
+
+
+def test_n4_is_the_4x4_path():
+    A = to_gpu(_logits(3000, 4, 3.0, 8))
+    assert torch.equal(api.birkhoff_fwd_n(A, "newton"), api.birkhoff_fwd(A, "newton"))
+    assert torch.equal(api.birkhoff_fwd_n(A, "newton_refined"), api.birkhoff_fwd(A, "newton_refined"))
+    assert torch.equal(api.birkhoff_fwd_n(A, "sinkhorn", 7), api.birkhoff_fwd(A, "sinkhorn", 7))
+
+
+def test_n_argument_errors():
+    L = api.lib()
+    A = torch.zeros((4, 3, 3), device=dev())
+    p = A.data_ptr()
+    assert L.mhc_birkhoff_fwd_n(p, p, 4, 9, 1, 0, None) == 3
+    assert L.mhc_birkhoff_fwd_n(p, p, 4, 0, 1, 0, None) == 3
+    assert L.mhc_birkhoff_fwd_n(p, p, 4, 3, 2, 0, None) == 4   # refined is 4 x 4 only
+    assert L.mhc_birkhoff_bwd_n(p, p, p, 4, 9, None) == 3
+    torch.cuda.synchronize()
