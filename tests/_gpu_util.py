@@ -34,8 +34,11 @@ def row_normalised(P):
 
 
 def per_matrix_rel_err(d, r):
-    d = np.asarray(d, np.float64).reshape(-1, 16)
-    r = np.asarray(r, np.float64).reshape(-1, 16)
+    d = np.asarray(d, np.float64)
+    r = np.asarray(r, np.float64)
+    # [count, n, n] or [count, n*n]: one matrix per leading index
+    d = d.reshape(d.shape[0], -1) if d.ndim >= 2 else d.reshape(-1, 16)
+    r = r.reshape(r.shape[0], -1) if r.ndim >= 2 else r.reshape(-1, 16)
     scale = np.abs(r).max(1)
     err = np.abs(d - r).max(1)
     return err / np.where(scale > 0, scale, 1.0), scale
