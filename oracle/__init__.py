@@ -49,10 +49,14 @@ def _load():
             lib.oracle_implicit_bwd.argtypes = [p, p, p, i64, i32]
             lib.oracle_mix_fwd.argtypes = [p, p, p, p, p, i64, i32, i64]
             lib.oracle_mix_bwd.argtypes = [p, p, p, p, p, p, p, p, p, i64, i32, i64]
+            lib.oracle_premap_fwd.argtypes = [p, p, p, i64, i32, i64]
+            lib.oracle_premap_bwd.argtypes = [p, p, p, p, p, i64, i32, i64]
+            lib.oracle_composite_gain.argtypes = [p, p, p, p, i64, i64, i32]
             lib.oracle_set_threads.argtypes = [i32]
             lib.oracle_get_threads.restype = i32
             for f in (lib.oracle_sinkhorn, lib.oracle_sinkhorn_bwd, lib.oracle_newton, lib.oracle_implicit_bwd,
-                      lib.oracle_mix_fwd, lib.oracle_mix_bwd):
+                      lib.oracle_mix_fwd, lib.oracle_mix_bwd, lib.oracle_premap_fwd, lib.oracle_premap_bwd,
+                      lib.oracle_composite_gain):
                 f.restype = i32
             _lib = lib
     return _lib
@@ -201,3 +205,44 @@ def mix_bwd(X_bf16, H, hpost, F_bf16, dY_bf16):
     if rc != 0:
         raise ValueError("oracle_mix_bwd: bad arguments")
     return dX, dH, dh, dF
+
+
+def premap_fwd(X_bf16, hpre_logits) -> np.ndarray:
+    """x_in[t,c] = sum_j sigmoid(hpre[t,j]) X[t,j,c] in double (forpes.ru mHC
+    explainer, "HC" and "mHC": pre-map back to the model width, non-negative
+    read weights through a sigmoid)."""
+    X = _u16(X_bf16)
+    T, n, C = X.shape
+    h = _f64(hpre_logits).reshape(T, n)
+    out = np.empty((T, C), dtype=np.float64)
+    if _load().oracle_premap_fwd(_ptr(X), _ptr(h), _ptr(out), T, n, C) != 0:
+        raise ValueError("oracle_premap_fwd: bad arguments")
+    return out
+
+
+def premap_bwd(X_bf16, hpre_logits, dx_in_bf16):
+    """Backward of premap_fwd: (dX, dhpre_logits) in double."""
+    X = _u16(X_bf16)
+    dx = _u16(dx_in_bf16)
+    T, n, C = X.shape
+    h = _f64(hpre_logits).reshape(T, n)
+    dX = np.empty((T, n, C), dtype=np.float64)
+    dh = np.empty((T, n), dtype=np.float64)
+    if _load().oracle_premap_bwd(_ptr(X), _ptr(h), _ptr(dx), _ptr(dX), _ptr(dh), T, n, C) != 0:
+        raise ValueError("oracle_premap_bwd: bad arguments")
+    return dX, dh
+
+
+def composite_gain(P_layers):
+    """Per-token product M = P_{L-1} ... P_0 of [L, T, n, n] matrices and its
+    largest absolute row sum and column sum (neo-ai mHC explainer: products of
+    doubly stochastic matrices stay doubly stochastic; finite Sinkhorn leaves a
+    gain above 1)."""
+    P = np.ascontiguousarray(np.asarray(P_layers, dtype=np.float64))
+    L, T, n, _ = P.shape
+    M = np.empty((T, n, n), dtype=np.float64)
+    gr = np.empty(T, dtype=np.float64)
+    gc = np.empty(T, dtype=np.float64)
+    if _load().oracle_composite_gain(_ptr(P), _ptr(M), _ptr(gr), _ptr(gc), L, T, n) != 0:
+        raise ValueError("oracle_composite_gain: bad arguments")
+    return M, gr, gc

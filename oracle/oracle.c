@@ -528,3 +528,92 @@ int oracle_mix_bwd(const uint16_t *X, const double *H, const double *hpost, cons
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* Pre-map (read map) and composite gain                              */
+/* ------------------------------------------------------------------ */
+
+static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+/* Pre-map of the widened residual back to the model width, with the read
+ * weights made non-negative by a sigmoid ([FP] "HC": before the layer the
+ * expanded representation is projected back to the model dimension; "mHC":
+ * the pre and post maps are made non-negative with a sigmoid):
+ *     x_in[t,c] = sum_j sigmoid(hpre[t,j]) X[t,j,c]. */
+int oracle_premap_fwd(const uint16_t *X, const double *hpre, double *x_in, int64_t T, int ns, int64_t C)
+{
+    if (T < 0 || C < 0 || ns < 1 || ns > ORACLE_NMAX) return -1;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t c = 0; c < C; ++c) {
+            double s = 0.0;
+            for (int j = 0; j < ns; ++j) s += sigmoid(hpre[t * ns + j]) * bf16_value(X[(t * ns + j) * C + c]);
+            x_in[t * C + c] = s;
+        }
+    return 0;
+}
+
+/* Its backward for upstream dx_in:
+ *     dX[t,j,c] = sigmoid(hpre[t,j]) dx_in[t,c]
+ *     dhpre[t,j] = sigmoid'(hpre[t,j]) sum_c dx_in[t,c] X[t,j,c]. */
+int oracle_premap_bwd(const uint16_t *X, const double *hpre, const uint16_t *dx_in, double *dX, double *dhpre,
+                      int64_t T, int ns, int64_t C)
+{
+    if (T < 0 || C < 0 || ns < 1 || ns > ORACLE_NMAX) return -1;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t t = 0; t < T; ++t)
+        for (int j = 0; j < ns; ++j) {
+            const double sg = sigmoid(hpre[t * ns + j]);
+            double acc = 0.0;
+            for (int64_t c = 0; c < C; ++c) {
+                const double g = bf16_value(dx_in[t * C + c]);
+                dX[(t * ns + j) * C + c] = sg * g;
+                acc += g * bf16_value(X[(t * ns + j) * C + c]);
+            }
+            dhpre[t * ns + j] = sg * (1.0 - sg) * acc;
+        }
+    return 0;
+}
+
+/* Composite mixing map across depth for each token: M = P_{L-1} ... P_1 P_0
+ * (layer 0 applied first), and its gains: the largest absolute row sum
+ * (how much the forward signal can grow) and the largest absolute column sum
+ * (the same for gradients).  A product of doubly stochastic matrices is
+ * doubly stochastic ([NA], compositional closure), so both gains are 1 for
+ * exact projections; inexact ones drift ([NA]: the ~1.6 gain of mHC is the
+ * residue of finite Sinkhorn iterations).  P_layers is [L][T][n][n]. */
+int oracle_composite_gain(const double *P_layers, double *M, double *gain_rows, double *gain_cols, int64_t L,
+                          int64_t T, int n)
+{
+    if (L < 1 || T < 0 || n < 1 || n > ORACLE_NMAX) return -1;
+    const int64_t nn = (int64_t)n * n;
+#pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t t = 0; t < T; ++t) {
+        double acc[ORACLE_NMAX * ORACLE_NMAX], tmp[ORACLE_NMAX * ORACLE_NMAX];
+        for (int64_t q = 0; q < nn; ++q) acc[q] = P_layers[t * nn + q];
+        for (int64_t l = 1; l < L; ++l) {
+            const double *Pl = P_layers + (l * T + t) * nn;
+            for (int i = 0; i < n; ++i)
+                for (int j = 0; j < n; ++j) {
+                    double s = 0.0;
+                    for (int k = 0; k < n; ++k) s += Pl[i * n + k] * acc[k * n + j];
+                    tmp[i * n + j] = s;
+                }
+            for (int64_t q = 0; q < nn; ++q) acc[q] = tmp[q];
+        }
+        double gr = 0.0, gc = 0.0;
+        for (int i = 0; i < n; ++i) {
+            double r = 0.0, c = 0.0;
+            for (int j = 0; j < n; ++j) {
+                r += fabs(acc[i * n + j]);
+                c += fabs(acc[j * n + i]);
+            }
+            if (r > gr) gr = r;
+            if (c > gc) gc = c;
+        }
+        for (int64_t q = 0; q < nn; ++q) M[t * nn + q] = acc[q];
+        gain_rows[t] = gr;
+        gain_cols[t] = gc;
+    }
+    return 0;
+}

@@ -141,3 +141,69 @@ def test_chained_gradient_through_projection(orc):
             lm = (dYv * orc.mix_fwd(X, orc.newton(Am, tol=1e-14), h, F)).sum((1, 2))
             fd[:, i, j] = (lp - lm) / (2 * eps)
     assert np.abs(dA - fd).max() <= 1e-6 * np.abs(fd).max() + 1e-8
+
+
+# ---------------------------------------------------------------- pre-map
+
+
+def test_premap_special_cases(orc):
+    X, _, _, _, _ = _case(T=3, C=32, seed=11)
+    T = X.shape[0]
+    # saturated read weights (sigmoid -> 1): the plain sum of the streams
+    big = np.full((T, 4), 60.0)
+    assert np.allclose(orc.premap_fwd(X, big), _bf16_value(X).sum(1), rtol=0, atol=1e-12)
+    # one stream read at weight 1/2 (logit 0), the others off (logit -> -inf)
+    for k in range(4):
+        h = np.full((T, 4), -800.0)
+        h[:, k] = 0.0
+        assert np.array_equal(orc.premap_fwd(X, h), 0.5 * _bf16_value(X)[:, k, :])
+
+
+def test_premap_bwd_is_adjoint_and_matches_finite_differences(orc):
+    X, _, dY, _, _ = _case(T=4, C=24, seed=12)
+    rng = np.random.default_rng(13)
+    h = rng.standard_normal((4, 4)) * 2
+    dx = dY[:, 0, :]
+    dX, dh = orc.premap_bwd(X, h, dx)
+    dxv = _bf16_value(dx)
+    # linear in X: <dx, premap(dirX)> = <dX, dirX>
+    dirX = _bf16_bits(rng.standard_normal(X.shape))
+    assert np.isclose((dxv * orc.premap_fwd(dirX, h)).sum(), (dX * _bf16_value(dirX)).sum(), rtol=1e-12)
+    # the read-map logits by central differences
+    eps = 1e-6
+    for j in range(4):
+        hp = h.copy()
+        hp[:, j] += eps
+        hm = h.copy()
+        hm[:, j] -= eps
+        fd = ((orc.premap_fwd(X, hp) - orc.premap_fwd(X, hm)) * dxv).sum(1) / (2 * eps)
+        assert np.allclose(dh[:, j], fd, rtol=1e-7, atol=1e-9)
+
+
+# ---------------------------------------------------------------- composite gain
+
+
+def test_composite_gain_pins(orc):
+    rng = np.random.default_rng(14)
+    L, T = 12, 50
+    A = rng.standard_normal((L * T, 4, 4)) * 3
+    P = orc.newton(A, tol=1e-13).reshape(L, T, 4, 4)
+    M, gr, gc = orc.composite_gain(P)
+    # exact projections compose to a doubly stochastic matrix: gains are 1
+    assert np.abs(gr - 1).max() < 1e-10 and np.abs(gc - 1).max() < 1e-10
+    # the product order: layer 0 is applied first (M = P_{L-1} ... P_0)
+    want = P[0]
+    for l in range(1, L):
+        want = P[l] @ want
+    assert np.abs(M - want).max() < 1e-12
+    # 20-round Sinkhorn ends on a column normalisation: every layer is column
+    # stochastic, so is their product (column gain 1), but the row sums are
+    # off one and the forward (row) gain drifts above 1
+    S = orc.sinkhorn(A * 3.0, 20).reshape(L, T, 4, 4)
+    _, gr_s, gc_s = orc.composite_gain(S)
+    assert np.abs(gc_s - 1).max() < 1e-9
+    assert gr_s.max() > 1.01
+    # permutation layers: composite is a permutation, gains exactly 1
+    perm = np.stack([np.eye(4)[rng.permutation(4)] for _ in range(L * T)]).reshape(L, T, 4, 4)
+    Mp, grp, gcp = orc.composite_gain(perm)
+    assert np.array_equal(grp, np.ones(T)) and set(np.unique(Mp)) <= {0.0, 1.0}
