@@ -58,6 +58,11 @@ def lib() -> ctypes.CDLL:
                 "mhc_sinkhorn_bwd": [p, p, p, i64, i32, p],
                 "mhc_birkhoff_fwd_n": [p, p, i64, i32, i32, i32, p],
                 "mhc_birkhoff_bwd_n": [p, p, p, i64, i32, p],
+                "mhc_premap_fwd": [p, p, p, i64, i64, p],
+                "mhc_premap_bwd": [p, p, p, p, p, i32, i64, i64, p],
+                "mhc_mix_post_bwd": [p, p, p, p, p, i64, i64, p],
+                "mhc_mix_premap_bwd": [p, p, p, p, p, p, p, p, p, i64, i64, p],
+                "mhc_composite_gain": [p, p, p, p, i64, i64, p],
                 "mhc_residual_mix_fwd": [p, p, p, p, p, i64, i64, p],
                 "mhc_residual_mix_bwd": [p, p, p, p, p, p, p, p, p, p, i64, i64, p],
                 "mhc_proj_mix_fwd": [p, p, p, p, p, p, i64, i64, i32, p],
@@ -267,6 +272,83 @@ def proj_mix_bwd(H_res, h_post, X, F, dY):
     _check(lib().mhc_proj_mix_bwd(_ptr(H_res), _ptr(h_post), _ptr(X), _ptr(F), _ptr(dY), _ptr(dX), _ptr(dl),
                                   _ptr(dh), _ptr(dF), T, C, _stream(X)))
     return dX, dl, dh, dF
+
+
+def premap_fwd(X, h_pre, out=None):
+    """x_in[t,c] = sum_j sigmoid(h_pre[t,j]) X[t,j,c] (bf16 in/out)."""
+    _need(X, "X", torch.bfloat16)
+    if X.dim() != 3 or X.shape[1] != 4:
+        raise ValueError("X must be [T, 4, C], got %s" % (tuple(X.shape),))
+    T, _, C = X.shape
+    _need(h_pre, "h_pre", torch.float32, (T, 4))
+    if out is None:
+        out = torch.empty((T, C), dtype=torch.bfloat16, device=X.device)
+    _need(out, "out", torch.bfloat16, (T, C))
+    _check(lib().mhc_premap_fwd(_ptr(X), _ptr(h_pre), _ptr(out), T, C, _stream(X)))
+    return out
+
+
+def premap_bwd(X, h_pre, dx_in, dX=None, accumulate=False):
+    """Backward of premap_fwd.  Returns (dX, dh_pre); with accumulate=True the
+    pre-map's contribution is added into the given dX."""
+    _need(X, "X", torch.bfloat16)
+    T, _, C = X.shape
+    _need(h_pre, "h_pre", torch.float32, (T, 4))
+    _need(dx_in, "dx_in", torch.bfloat16, (T, C))
+    if dX is None:
+        if accumulate:
+            raise ValueError("accumulate needs dX")
+        dX = torch.empty_like(X)
+    _need(dX, "dX", torch.bfloat16, X.shape)
+    dh = torch.empty_like(h_pre)
+    _check(lib().mhc_premap_bwd(_ptr(X), _ptr(h_pre), _ptr(dx_in), _ptr(dX), _ptr(dh), 1 if accumulate else 0,
+                                T, C, _stream(X)))
+    return dX, dh
+
+
+def mix_post_bwd(dY, F, h_post):
+    """First half of the split mix backward: (dF, dh_post)."""
+    _need(dY, "dY", torch.bfloat16)
+    T, _, C = dY.shape
+    _need(F, "F", torch.bfloat16, (T, C))
+    _need(h_post, "h_post", torch.float32, (T, 4))
+    dF = torch.empty_like(F)
+    dh = torch.empty_like(h_post)
+    _check(lib().mhc_mix_post_bwd(_ptr(dY), _ptr(F), _ptr(h_post), _ptr(dF), _ptr(dh), T, C, _stream(dY)))
+    return dF, dh
+
+
+def mix_premap_bwd(X, H_res, h_pre, dY, dx_in, need_dH=False, need_dlogits=True):
+    """Second half of the split mix backward, fused with the pre-map backward:
+    dX = H_res^T dY + sigmoid(h_pre) dx_in, dh_pre, and optionally dH_res and the
+    chained dlogits.  Returns a dict."""
+    _need(X, "X", torch.bfloat16)
+    T, _, C = X.shape
+    _need(H_res, "H_res", torch.float32, (T, 4, 4))
+    _need(h_pre, "h_pre", torch.float32, (T, 4))
+    _need(dY, "dY", torch.bfloat16, X.shape)
+    _need(dx_in, "dx_in", torch.bfloat16, (T, C))
+    dX = torch.empty_like(X)
+    dhp = torch.empty_like(h_pre)
+    dH = torch.empty_like(H_res) if need_dH else None
+    dl = torch.empty_like(H_res) if need_dlogits else None
+    _check(lib().mhc_mix_premap_bwd(_ptr(X), _ptr(H_res), _ptr(h_pre), _ptr(dY), _ptr(dx_in), _ptr(dX), _ptr(dH),
+                                    _ptr(dhp), _ptr(dl), T, C, _stream(X)))
+    return {"dX": dX, "dh_pre": dhp, "dH_res": dH, "dlogits": dl}
+
+
+def composite_gain(P_layers, need_M=True):
+    """Per-token product across depth of [L, T, 4, 4] matrices and its row and
+    column gains.  Returns (M or None, gain_rows, gain_cols)."""
+    _need(P_layers, "P_layers", torch.float32)
+    if P_layers.dim() != 4 or tuple(P_layers.shape[-2:]) != (4, 4):
+        raise ValueError("P_layers must be [L, T, 4, 4]")
+    L, T = int(P_layers.shape[0]), int(P_layers.shape[1])
+    M = torch.empty((T, 4, 4), dtype=torch.float32, device=P_layers.device) if need_M else None
+    gr = torch.empty(T, dtype=torch.float32, device=P_layers.device)
+    gc = torch.empty_like(gr)
+    _check(lib().mhc_composite_gain(_ptr(P_layers), _ptr(M), _ptr(gr), _ptr(gc), L, T, _stream(P_layers)))
+    return M, gr, gc
 
 
 class BirkhoffProjection(torch.autograd.Function):

@@ -38,4 +38,16 @@ cudaError_t launch_proj_mix_fwd(const float* logits, const float* hpost, const u
                                 const uint16_t* F, uint16_t* Y, float* H, int64_t T, int64_t C,
                                 int maxit, cudaStream_t s);
 
+cudaError_t launch_premap_fwd(const uint16_t* X, const float* hpre, uint16_t* x_in, int64_t T, int64_t C,
+                              cudaStream_t s);
+cudaError_t launch_premap_bwd(const uint16_t* X, const float* hpre, const uint16_t* dx_in, uint16_t* dX,
+                              float* dhpre, bool accumulate, int64_t T, int64_t C, cudaStream_t s);
+cudaError_t launch_mix_post_bwd(const uint16_t* dY, const uint16_t* F, const float* hpost, uint16_t* dF,
+                                float* dhpost, int64_t T, int64_t C, cudaStream_t s);
+cudaError_t launch_mix_premap_bwd(const uint16_t* X, const float* H, const float* hpre, const uint16_t* dY,
+                                  const uint16_t* dx_in, uint16_t* dX, float* dH, float* dhpre, float* dlogits,
+                                  int64_t T, int64_t C, cudaStream_t s);
+cudaError_t launch_composite_gain(const float* P, float* M, float* gain_rows, float* gain_cols, int64_t L, int64_t T,
+                                  cudaStream_t s);
+
 }  // namespace mhc

@@ -201,4 +201,66 @@ int mhc_proj_mix_bwd(const float* H_res, const float* h_post, const uint16_t* X,
                                            static_cast<cudaStream_t>(stream)));
 }
 
+int mhc_premap_fwd(const uint16_t* X, const float* h_pre, uint16_t* x_in, int64_t T, int64_t C, void* stream)
+{
+    int rc = check_mix_sizes(T, C);
+    if (rc != MHC_OK) return rc;
+    if (T == 0) return MHC_OK;
+    if (!X || !h_pre || !x_in) return MHC_ERR_NULL;
+    if (misaligned(X) || misaligned(h_pre) || misaligned(x_in)) return MHC_ERR_ALIGN;
+    return cuda_status(mhc::launch_premap_fwd(X, h_pre, x_in, T, C, static_cast<cudaStream_t>(stream)));
+}
+
+int mhc_premap_bwd(const uint16_t* X, const float* h_pre, const uint16_t* dx_in, uint16_t* dX, float* dh_pre,
+                   int accumulate, int64_t T, int64_t C, void* stream)
+{
+    int rc = check_mix_sizes(T, C);
+    if (rc != MHC_OK) return rc;
+    if (accumulate != 0 && accumulate != 1) return MHC_ERR_ARG;
+    if (T == 0) return MHC_OK;
+    if (!X || !h_pre || !dx_in || !dX || !dh_pre) return MHC_ERR_NULL;
+    if (misaligned(X) || misaligned(h_pre) || misaligned(dx_in) || misaligned(dX) || misaligned(dh_pre))
+        return MHC_ERR_ALIGN;
+    return cuda_status(mhc::launch_premap_bwd(X, h_pre, dx_in, dX, dh_pre, accumulate == 1, T, C,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+int mhc_mix_post_bwd(const uint16_t* dY, const uint16_t* F, const float* h_post, uint16_t* dF, float* dh_post,
+                     int64_t T, int64_t C, void* stream)
+{
+    int rc = check_mix_sizes(T, C);
+    if (rc != MHC_OK) return rc;
+    if (T == 0) return MHC_OK;
+    if (!dY || !F || !h_post || !dF || !dh_post) return MHC_ERR_NULL;
+    if (misaligned(dY) || misaligned(F) || misaligned(h_post) || misaligned(dF) || misaligned(dh_post))
+        return MHC_ERR_ALIGN;
+    return cuda_status(mhc::launch_mix_post_bwd(dY, F, h_post, dF, dh_post, T, C, static_cast<cudaStream_t>(stream)));
+}
+
+int mhc_mix_premap_bwd(const uint16_t* X, const float* H_res, const float* h_pre, const uint16_t* dY,
+                       const uint16_t* dx_in, uint16_t* dX, float* dH_res, float* dh_pre, float* dlogits, int64_t T,
+                       int64_t C, void* stream)
+{
+    int rc = check_mix_sizes(T, C);
+    if (rc != MHC_OK) return rc;
+    if (T == 0) return MHC_OK;
+    if (!X || !H_res || !h_pre || !dY || !dx_in || !dX || !dh_pre) return MHC_ERR_NULL;
+    if (misaligned(X) || misaligned(H_res) || misaligned(h_pre) || misaligned(dY) || misaligned(dx_in) ||
+        misaligned(dX) || misaligned(dH_res) || misaligned(dh_pre) || misaligned(dlogits))
+        return MHC_ERR_ALIGN;
+    return cuda_status(mhc::launch_mix_premap_bwd(X, H_res, h_pre, dY, dx_in, dX, dH_res, dh_pre, dlogits, T, C,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
+int mhc_composite_gain(const float* P_layers, float* M, float* gain_rows, float* gain_cols, int64_t L, int64_t T,
+                       void* stream)
+{
+    if (L < 1 || T < 0 || L > (int64_t(1) << 20) || T > (int64_t(1) << 36)) return MHC_ERR_SIZE;
+    if (T == 0) return MHC_OK;
+    if (!P_layers || !gain_rows || !gain_cols) return MHC_ERR_NULL;
+    if (misaligned(P_layers) || misaligned(M)) return MHC_ERR_ALIGN;
+    return cuda_status(
+        mhc::launch_composite_gain(P_layers, M, gain_rows, gain_cols, L, T, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

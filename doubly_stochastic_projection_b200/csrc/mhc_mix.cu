@@ -14,10 +14,9 @@
 // vectors (8 bf16 channels) of each stream with streaming (evict-first)
 // loads and stores, so each warp touches 512 contiguous bytes per stream per
 // instruction.  The per-token H and h_post are broadcast loads.
-#include <cuda_bf16.h>
-
 #include "birkhoff_math.cuh"
 #include "launch.h"
+#include "mix_common.cuh"
 
 namespace mhc {
 
@@ -26,40 +25,6 @@ namespace {
 constexpr int kMixThreads = 128;
 constexpr int kMixWarps = kMixThreads / 32;
 constexpr int kFusedTok = 4;  // tokens projected together per CTA round
-
-__device__ __forceinline__ void unpack8(const uint4 v, float (&f)[8])
-{
-    f[0] = __uint_as_float(v.x << 16);
-    f[1] = __uint_as_float(v.x & 0xffff0000u);
-    f[2] = __uint_as_float(v.y << 16);
-    f[3] = __uint_as_float(v.y & 0xffff0000u);
-    f[4] = __uint_as_float(v.z << 16);
-    f[5] = __uint_as_float(v.z & 0xffff0000u);
-    f[6] = __uint_as_float(v.w << 16);
-    f[7] = __uint_as_float(v.w & 0xffff0000u);
-}
-
-__device__ __forceinline__ uint32_t pack2(float lo, float hi)
-{
-    const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);  // round to nearest even
-    return *reinterpret_cast<const uint32_t*>(&b);
-}
-
-__device__ __forceinline__ uint4 pack8(const float (&f)[8])
-{
-    return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
-}
-
-__device__ __forceinline__ void load_maps(const float* H, const float* hpost, int64_t t, float (&h)[16],
-                                          float (&hp)[4])
-{
-    load16(H + 16 * t, h);
-    const float4 q = __ldg(reinterpret_cast<const float4*>(hpost) + t);
-    hp[0] = q.x;
-    hp[1] = q.y;
-    hp[2] = q.z;
-    hp[3] = q.w;
-}
 
 // One 8-channel vector of one token: y_i = sum_j h_ij x_j + hp_i f.
 __device__ __forceinline__ void mix_vec(const float (&h)[16], const float (&hp)[4], const uint4 (&x)[4],
@@ -160,13 +125,6 @@ proj_mix_fwd_kernel(const float* logits, const float* hpost, const uint4* X, con
         }
         __syncthreads();
     }
-}
-
-__device__ __forceinline__ float warp_sum(float v)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
 }
 
 // One 8-channel vector of the backward: dX, dF out; dH, dh_post partial sums.

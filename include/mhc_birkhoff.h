@@ -247,6 +247,68 @@ MHC_API int mhc_proj_mix_bwd(const float *H_res, const float *h_post, const uint
                      const uint16_t *F, const uint16_t *dY, uint16_t *dX, float *dlogits,
                      float *dh_post, uint16_t *dF, int64_t T, int64_t C, void *stream);
 
+/*
+ * mhc_premap_fwd -- the read map (pre-map) that projects the widened residual
+ * back to the model width before the layer, with non-negative weights through
+ * a sigmoid ([FP] "HC" and "mHC"):
+ *     x_in[t,c] = sum_j sigmoid(h_pre[t,j]) X[t,j,c]
+ *
+ *   X [T][4][C] bf16, read.  h_pre [T][4] float, read: the logits of the read
+ *   weights (the sigmoid is applied here).  x_in [T][C] bf16, written.
+ */
+MHC_API int mhc_premap_fwd(const uint16_t *X, const float *h_pre, uint16_t *x_in, int64_t T, int64_t C,
+                           void *stream);
+
+/*
+ * mhc_premap_bwd -- backward of mhc_premap_fwd for upstream dx_in:
+ *     dX[t,j,c] (+)= s_j dx_in[t,c],   dh_pre[t,j] = s_j (1 - s_j) sum_c dx_in[t,c] X[t,j,c]
+ * with s_j = sigmoid(h_pre[t,j]).  accumulate = 1 adds into dX (read and
+ * rewritten, e.g. the mix backward's dX); 0 overwrites it.
+ *
+ *   dx_in [T][C] bf16, read.  dX [T][4][C] bf16, written (read too when
+ *   accumulating).  dh_pre [T][4] float, written.
+ */
+MHC_API int mhc_premap_bwd(const uint16_t *X, const float *h_pre, const uint16_t *dx_in, uint16_t *dX,
+                           float *dh_pre, int accumulate, int64_t T, int64_t C, void *stream);
+
+/*
+ * The residual-mix backward split in two, so that one pass over X serves the
+ * mix and the pre-map (in a layer's backward dx_in is only known after the
+ * layer's own backward, which needs dF first):
+ *
+ * mhc_mix_post_bwd -- the part that needs only dY and F:
+ *     dF[t,c] = sum_i h_post[t,i] dY[t,i,c],   dh_post[t,i] = sum_c dY[t,i,c] F[t,c]
+ *
+ * mhc_mix_premap_bwd -- the rest, together with the pre-map's backward:
+ *     dX[t,j,c]   = sum_i H_res[t,i,j] dY[t,i,c] + s_j dx_in[t,c]
+ *     dH_res[t,i,j] = sum_c dY[t,i,c] X[t,j,c]          (written if non-NULL)
+ *     dh_pre[t,j] = s_j (1 - s_j) sum_c dx_in[t,c] X[t,j,c]
+ *     dlogits = implicit backward of the projection at P = H_res, dP = dH_res
+ *               (written if non-NULL; H_res must be the Newton projection)
+ * Together they move 38 C bytes per token; mhc_residual_mix_bwd followed by
+ * mhc_premap_bwd with accumulate = 1 moves 54 C.
+ */
+MHC_API int mhc_mix_post_bwd(const uint16_t *dY, const uint16_t *F, const float *h_post, uint16_t *dF,
+                             float *dh_post, int64_t T, int64_t C, void *stream);
+MHC_API int mhc_mix_premap_bwd(const uint16_t *X, const float *H_res, const float *h_pre, const uint16_t *dY,
+                               const uint16_t *dx_in, uint16_t *dX, float *dH_res, float *dh_pre,
+                               float *dlogits, int64_t T, int64_t C, void *stream);
+
+/*
+ * mhc_composite_gain -- diagnostic of the composite mixing map across depth:
+ * per token, M = P_{L-1} ... P_1 P_0 (layer 0 applied first) and its largest
+ * absolute row sum (forward signal gain) and column sum (gradient gain).
+ * Products of doubly stochastic matrices are doubly stochastic ([NA],
+ * compositional closure), so both gains are 1 for exact projections; [NA]
+ * attributes mHC's measured ~1.6 gain to the residue of finite Sinkhorn
+ * iterations.
+ *
+ *   P_layers [L][T][4][4] float, read.  M [T][4][4] float, written, or NULL.
+ *   gain_rows, gain_cols [T] float, written.  L >= 1.
+ */
+MHC_API int mhc_composite_gain(const float *P_layers, float *M, float *gain_rows, float *gain_cols, int64_t L,
+                               int64_t T, void *stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 MHC_API const char *mhc_status_string(int status);
 
