@@ -388,7 +388,42 @@ def extras(dev, stream, flush, hbm, api, inputs):
             "fused_bwd_gbs": bfb / tfb / 1e9, "fused_bwd_frac_hbm": bfb / tfb / 1e9 / hbm,
             "fused_fwd_bwd_tokens_per_s": T / (tff + tfb),
         })
-        del m, X, F, dY, Y, H, lg, h
+        # read map and the split backward (dF, dh_post first; then dX with the
+        # pre-map's contribution, dH, dh_pre and dlogits in one pass over X)
+        hpre = torch.from_numpy(inputs.birkhoff_logits(T, "normal1", 14)[:, 0, :].copy()).to(dev)
+        dx_in = inputs.bf16_normal((T, C), 15, dev)
+        x_in = torch.empty_like(F)
+        tp = event_time(lambda: api.premap_fwd(X, hpre, out=x_in), reps, stream, flush)
+        t_split = event_time(lambda: (api.mix_post_bwd(dY, F, h),
+                                      api.mix_premap_bwd(X, H, hpre, dY, dx_in, need_dlogits=True)), reps, stream, flush)
+        def unsplit():
+            o = api.residual_mix_bwd(X, H, h, F, dY, need_dlogits=True)
+            api.premap_bwd(X, hpre, dx_in, dX=o["dX"], accumulate=True)
+        t_unsplit = event_time(unsplit, reps, stream, flush)
+        bp = (10 * C + 16) * T
+        out["mix"][-1].update({
+            "premap_fwd_gbs": bp / tp / 1e9, "premap_fwd_frac_hbm": bp / tp / 1e9 / hbm,
+            "split_bwd_with_premap_us": t_split * 1e6, "unsplit_bwd_then_premap_bwd_us": t_unsplit * 1e6,
+            "split_bwd_gbs": (38 * C + 240) * T / t_split / 1e9,
+            "split_bwd_frac_hbm": (38 * C + 240) * T / t_split / 1e9 / hbm})
+        del m, X, F, dY, Y, H, lg, h, hpre, dx_in, x_in
+        torch.cuda.empty_cache()
+    # composite gain across 60 layers (the amax-gain drift of finite Sinkhorn)
+    out["composite_gain"] = []
+    Lg, Tg = 60, 65536
+    for dist in ("normal1", "normal3", "normal10"):
+        A = torch.from_numpy(inputs.birkhoff_logits(Lg * Tg, dist, 16)).to(dev)
+        row = {"layers": Lg, "tokens": Tg, "dist": dist}
+        for method, iters in (("newton", 0), ("sinkhorn", 20)):
+            P = api.birkhoff_fwd(A, method, iters).reshape(Lg, Tg, 4, 4)
+            _, gr, gc = api.composite_gain(P, need_M=False)
+            tg = event_time(lambda: api.composite_gain(P, need_M=False), reps, stream, flush)
+            row[method] = {"row_gain_max": float(gr.max()), "row_gain_p99": float(torch.quantile(gr, 0.99)),
+                           "col_gain_max": float(gc.max())}
+            row["kernel_gbs"] = Lg * Tg * 64 / tg / 1e9
+            del P
+        out["composite_gain"].append(row)
+        del A
         torch.cuda.empty_cache()
     return out
 
