@@ -14,6 +14,7 @@
 
 #include "birkhoff_math.cuh"
 #include "launch.h"
+#include "pdl.cuh"
 
 namespace mhc {
 
@@ -30,6 +31,8 @@ constexpr int kProjThreadsSmall = 128;
 __global__ void __launch_bounds__(kProjThreads)
 sinkhorn_fwd_kernel(const float* logits, float* P, int64_t n, int iters)
 {
+    pdl_wait();
+    pdl_trigger();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
         float a[16];
@@ -43,6 +46,8 @@ template <bool kDiag, bool kRefine>
 __global__ void __launch_bounds__(kProjThreads)
 newton_fwd_kernel(const float* logits, float* P, int32_t* iters_out, int64_t n, int maxit)
 {
+    pdl_wait();
+    pdl_trigger();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
         float a[16];
@@ -59,6 +64,8 @@ template <bool kRecompute>
 __global__ void __launch_bounds__(kProjThreads)
 implicit_bwd_kernel(const float* logits, const float* P, const float* dP, float* dlogits, int64_t n)
 {
+    pdl_wait();
+    pdl_trigger();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
         float p[16], g[16], out[16];
@@ -77,6 +84,8 @@ implicit_bwd_kernel(const float* logits, const float* P, const float* dP, float*
 __global__ void __launch_bounds__(kProjThreads)
 sinkhorn_bwd_kernel(const float* logits, const float* dP, float* dlogits, int64_t n, int iters)
 {
+    pdl_wait();
+    pdl_trigger();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
         float a[16], g[16], out[16];
@@ -134,32 +143,25 @@ int persistent_grid(const void* kernel, int threads, size_t smem, int64_t blocks
 cudaError_t launch_sinkhorn_fwd(const float* logits, float* P, int64_t n, int iters, cudaStream_t s)
 {
     const Launch L = projection_launch((const void*)sinkhorn_fwd_kernel, n);
-    sinkhorn_fwd_kernel<<<L.grid, L.threads, 0, s>>>(logits, P, n, iters);
-    return cudaGetLastError();
+    return launch_pdl(sinkhorn_fwd_kernel, L.grid, L.threads, 0, s, logits, P, n, iters);
 }
 
 template <bool kDiag, bool kRefine>
-static void launch_newton(const float* logits, float* P, int32_t* iters_out, int64_t n, int maxit, cudaStream_t s)
+static cudaError_t launch_newton(const float* logits, float* P, int32_t* iters_out, int64_t n, int maxit,
+                                 cudaStream_t s)
 {
     const Launch L = projection_launch((const void*)newton_fwd_kernel<kDiag, kRefine>, n);
-    newton_fwd_kernel<kDiag, kRefine><<<L.grid, L.threads, 0, s>>>(logits, P, iters_out, n, maxit);
+    return launch_pdl(newton_fwd_kernel<kDiag, kRefine>, L.grid, L.threads, 0, s, logits, P, iters_out, n, maxit);
 }
 
 cudaError_t launch_newton_fwd(const float* logits, float* P, int32_t* iters_out, int64_t n, int maxit,
                               bool refine, cudaStream_t s)
 {
-    if (iters_out) {
-        if (refine)
-            launch_newton<true, true>(logits, P, iters_out, n, maxit, s);
-        else
-            launch_newton<true, false>(logits, P, iters_out, n, maxit, s);
-    } else {
-        if (refine)
-            launch_newton<false, true>(logits, P, nullptr, n, maxit, s);
-        else
-            launch_newton<false, false>(logits, P, nullptr, n, maxit, s);
-    }
-    return cudaGetLastError();
+    if (iters_out)
+        return refine ? launch_newton<true, true>(logits, P, iters_out, n, maxit, s)
+                      : launch_newton<true, false>(logits, P, iters_out, n, maxit, s);
+    return refine ? launch_newton<false, true>(logits, P, nullptr, n, maxit, s)
+                  : launch_newton<false, false>(logits, P, nullptr, n, maxit, s);
 }
 
 cudaError_t launch_implicit_bwd(const float* logits, const float* P, const float* dP, float* dlogits,
@@ -167,20 +169,19 @@ cudaError_t launch_implicit_bwd(const float* logits, const float* P, const float
 {
     if (P) {
         const Launch L = projection_launch((const void*)implicit_bwd_kernel<false>, n);
-        implicit_bwd_kernel<false><<<L.grid, L.threads, 0, s>>>(nullptr, P, dP, dlogits, n);
-    } else {
-        const Launch L = projection_launch((const void*)implicit_bwd_kernel<true>, n);
-        implicit_bwd_kernel<true><<<L.grid, L.threads, 0, s>>>(logits, nullptr, dP, dlogits, n);
+        return launch_pdl(implicit_bwd_kernel<false>, L.grid, L.threads, 0, s, (const float*)nullptr, P, dP,
+                          dlogits, n);
     }
-    return cudaGetLastError();
+    const Launch L = projection_launch((const void*)implicit_bwd_kernel<true>, n);
+    return launch_pdl(implicit_bwd_kernel<true>, L.grid, L.threads, 0, s, logits, (const float*)nullptr, dP,
+                      dlogits, n);
 }
 
 cudaError_t launch_sinkhorn_bwd(const float* logits, const float* dP, float* dlogits, int64_t n, int iters,
                                 cudaStream_t s)
 {
     const Launch L = projection_launch((const void*)sinkhorn_bwd_kernel, n);
-    sinkhorn_bwd_kernel<<<L.grid, L.threads, 0, s>>>(logits, dP, dlogits, n, iters);
-    return cudaGetLastError();
+    return launch_pdl(sinkhorn_bwd_kernel, L.grid, L.threads, 0, s, logits, dP, dlogits, n, iters);
 }
 
 }  // namespace mhc

@@ -5,6 +5,7 @@
 // 4 x 4 kernels.
 #include "birkhoff_math_n.cuh"
 #include "launch.h"
+#include "pdl.cuh"
 
 namespace mhc {
 
@@ -30,6 +31,8 @@ template <int N>
 __global__ void __launch_bounds__(kThreadsN)
 sinkhorn_fwd_n_kernel(const float* logits, float* P, int64_t n, int iters)
 {
+    pdl_wait();
+    pdl_trigger();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
         float a[N * N];
@@ -43,6 +46,8 @@ template <int N>
 __global__ void __launch_bounds__(kThreadsN)
 newton_fwd_n_kernel(const float* logits, float* P, int64_t n, int maxit)
 {
+    pdl_wait();
+    pdl_trigger();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
         float a[N * N];
@@ -56,6 +61,8 @@ template <int N>
 __global__ void __launch_bounds__(kThreadsN)
 implicit_bwd_n_kernel(const float* P, const float* dP, float* dlogits, int64_t n)
 {
+    pdl_wait();
+    pdl_trigger();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride)
         implicit_vjp_n<N>(P + (int64_t)N * N * m, dP + (int64_t)N * N * m, dlogits + (int64_t)N * N * m);
@@ -67,12 +74,10 @@ cudaError_t launch_fwd_n(const float* logits, float* P, int64_t n, bool newton, 
     const int64_t blocks = (n + kThreadsN - 1) / kThreadsN;
     if (newton) {
         const int grid = persistent_grid((const void*)newton_fwd_n_kernel<N>, kThreadsN, 0, blocks);
-        newton_fwd_n_kernel<N><<<grid, kThreadsN, 0, s>>>(logits, P, n, iters);
-    } else {
-        const int grid = persistent_grid((const void*)sinkhorn_fwd_n_kernel<N>, kThreadsN, 0, blocks);
-        sinkhorn_fwd_n_kernel<N><<<grid, kThreadsN, 0, s>>>(logits, P, n, iters);
+        return launch_pdl(newton_fwd_n_kernel<N>, grid, kThreadsN, 0, s, logits, P, n, iters);
     }
-    return cudaGetLastError();
+    const int grid = persistent_grid((const void*)sinkhorn_fwd_n_kernel<N>, kThreadsN, 0, blocks);
+    return launch_pdl(sinkhorn_fwd_n_kernel<N>, grid, kThreadsN, 0, s, logits, P, n, iters);
 }
 
 template <int N>
@@ -80,8 +85,7 @@ cudaError_t launch_bwd_n(const float* P, const float* dP, float* dlogits, int64_
 {
     const int64_t blocks = (n + kThreadsN - 1) / kThreadsN;
     const int grid = persistent_grid((const void*)implicit_bwd_n_kernel<N>, kThreadsN, 0, blocks);
-    implicit_bwd_n_kernel<N><<<grid, kThreadsN, 0, s>>>(P, dP, dlogits, n);
-    return cudaGetLastError();
+    return launch_pdl(implicit_bwd_n_kernel<N>, grid, kThreadsN, 0, s, P, dP, dlogits, n);
 }
 
 }  // namespace

@@ -83,7 +83,7 @@ def _run_case(orc, name, T, C, n_sample=None, seed=0):
     _rel_ok(to_np64(Y2[idx]), ref, MIX_REL_TOL)
 
 
-@pytest.mark.parametrize("T,C", [(1, 8), (3, 1040), (17, 4096), (5, 7168), (64, 8 * 129)])
+@pytest.mark.parametrize("T,C", [(1, 8), (3, 1040), (17, 4096), (5, 7168), (64, 8 * 129), (1000, 8 * 385)])
 def test_mix_small_and_ragged(orc, T, C):
     _run_case(orc, "mix_T16384_C4096", T, C)
 

@@ -27,7 +27,8 @@ def _case(T, C, seed):
     return m, h_pre, dx_in
 
 
-@pytest.mark.parametrize("T,C,n_sample", [(1, 8, None), (5, 1040, None), (33, 4096, None), (16384, 4096, 24)])
+@pytest.mark.parametrize("T,C,n_sample", [(1, 8, None), (5, 1040, None), (33, 4096, None), (1000, 8 * 385, None),
+                                         (16384, 4096, 24)])
 def test_premap_and_split_backward(orc, T, C, n_sample):
     m, h_pre, dx_in = _case(T, C, 40)
     X, F, dY = m["X"], m["F"], m["dY"]
