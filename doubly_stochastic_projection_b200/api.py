@@ -56,6 +56,7 @@ def lib() -> ctypes.CDLL:
                 "mhc_birkhoff_fwd_diag": [p, p, p, i64, i32, p],
                 "mhc_birkhoff_bwd": [p, p, p, p, i64, p],
                 "mhc_sinkhorn_bwd": [p, p, p, i64, i32, p],
+                "mhc_exp_shifted": [p, p, i64, p],
                 "mhc_birkhoff_fwd_n": [p, p, i64, i32, i32, i32, p],
                 "mhc_birkhoff_bwd_n": [p, p, p, i64, i32, p],
                 "mhc_premap_fwd": [p, p, p, i64, i64, p],
@@ -190,6 +191,16 @@ def birkhoff_bwd_n(dP: torch.Tensor, P: torch.Tensor, out: torch.Tensor | None =
         out = torch.empty_like(dP)
     _need(out, "out", torch.float32, dP.shape)
     _check(lib().mhc_birkhoff_bwd_n(_ptr(P), _ptr(dP), _ptr(out), count, n, _stream(dP)))
+    return out
+
+
+def exp_shifted(x, out=None):
+    """e^x as the projection kernels evaluate it for max-shifted logits (x <= 0)."""
+    _need(x, "x", torch.float32)
+    if out is None:
+        out = torch.empty_like(x)
+    _need(out, "out", torch.float32, x.shape)
+    _check(lib().mhc_exp_shifted(_ptr(x), _ptr(out), x.numel(), _stream(x)))
     return out
 
 

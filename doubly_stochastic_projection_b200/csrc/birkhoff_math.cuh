@@ -47,6 +47,29 @@ __device__ __forceinline__ float rcp_approx(float x)
     return y;
 }
 
+// e^x for the max-shifted logits (x <= 0), by the argument split of Cody and
+// Waite (Software Manual for the Elementary Functions, 1980): x log2(e) is
+// written t + r, t the fp32 product and r its rounding error recovered by an
+// fma (plus the low part of log2 e), so e^x = 2^t 2^r with 2^t from the
+// hardware base-2 exponential (ex2.approx, subnormal results flushed to zero)
+// and 2^r = 1 + r ln 2 to first order (|r| < 2e-5 for x > -110, so the
+// neglected term is below 1e-10 relative).  A handful of instructions where
+// the library expf spends several times as many; the start-up of the Newton
+// solver exponentiates all sixteen entries.  x = -inf gives NaN (the fma of
+// -inf and +inf), which the solvers report as a non-finite logit; x = 0 gives
+// exactly 1.
+__device__ __forceinline__ float exp_shifted(float x)
+{
+    constexpr float kLog2eHi = 1.44269502162933349609375f;  // log2(e) rounded to fp32
+    constexpr float kLog2eLo = 1.925962991126617468e-8f;    // log2(e) - kLog2eHi
+    constexpr float kLn2 = 0.6931471805599453094f;
+    const float t = x * kLog2eHi;
+    const float r = fmaf(x, kLog2eLo, fmaf(x, kLog2eHi, -t));
+    float p;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(p) : "f"(t));
+    return fmaf(p, r * kLn2, p);
+}
+
 __device__ __forceinline__ void load16(const float* p, float (&a)[16])
 {
     const float4* q = reinterpret_cast<const float4*>(p);
@@ -186,13 +209,13 @@ __device__ __forceinline__ bool laplacian_solve(const PairWeights& w, float r0, 
 // K = exp(A - rowmax A) ([BA] §2.1 max shift), then `iters` rounds of
 // "divide every row by its sum, then every column by its sum" ([DS]; [BA] §1
 // names 20 as the usual fixed count).  Division is done as multiplication by
-// a correctly rounded reciprocal.
+// a reciprocal within 1 ulp (rcp_approx).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void sinkhorn_project(float (&a)[16], int iters)
 {
     shift_rows_by_max(a);
 #pragma unroll
-    for (int k = 0; k < 16; ++k) a[k] = expf(a[k]);
+    for (int k = 0; k < 16; ++k) a[k] = exp_shifted(a[k]);
     for (int it = 0; it < iters; ++it) {
         normalize_rows(a);
         normalize_cols(a);
@@ -300,7 +323,7 @@ __device__ __forceinline__ void sinkhorn_vjp(const float (&A)[16], const float (
     }
     shift_rows_by_max(K);
 #pragma unroll
-    for (int k = 0; k < 16; ++k) K[k] = expf(K[k]);
+    for (int k = 0; k < 16; ++k) K[k] = exp_shifted(K[k]);
 
     const int nseg = (iters + kSkSegment - 1) / kSkSegment;
     for (int seg = nseg - 1; seg >= 0; --seg) {
@@ -398,7 +421,7 @@ __device__ __forceinline__ int newton_project(float (&a)[16], int maxit)
     shift_rows_by_max(a);
     shift_cols_by_max(a);
 #pragma unroll
-    for (int k = 0; k < 16; ++k) a[k] = expf(a[k]);
+    for (int k = 0; k < 16; ++k) a[k] = exp_shifted(a[k]);
     // one Sinkhorn round (columns, then rows) as the warm start; every row and
     // column of exp(A) now holds a 1, so no sum is below one
     normalize_cols(a);
@@ -437,8 +460,8 @@ __device__ __forceinline__ int newton_project(float (&a)[16], int maxit)
             d2 *= sc;
         }
         // Column factors e^{t d_j}.  Their rounding only perturbs the step,
-        // never the fixed point, so the fast exponential is used here (the
-        // exponential of the logits above is the exact one).
+        // never the fixed point, so the plain fast exponential is used here
+        // (the logits themselves go through the compensated exp_shifted).
         float e0 = __expf(d0), e1 = __expf(d1), e2 = __expf(d2);
         float s[4];
 #pragma unroll

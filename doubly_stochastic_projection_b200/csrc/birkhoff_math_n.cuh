@@ -122,7 +122,7 @@ __device__ __forceinline__ void sinkhorn_project_n(float (&a)[N * N], int iters)
 {
     shift_rows_by_max_n<N>(a);
 #pragma unroll
-    for (int k = 0; k < N * N; ++k) a[k] = expf(a[k]);
+    for (int k = 0; k < N * N; ++k) a[k] = exp_shifted(a[k]);
     for (int it = 0; it < iters; ++it) {
         normalize_rows_n<N>(a);
         normalize_cols_n<N>(a);
@@ -143,7 +143,7 @@ __device__ __forceinline__ int newton_project_n(float (&a)[N * N], int maxit)
     shift_rows_by_max_n<N>(a);
     shift_cols_by_max_n<N>(a);
 #pragma unroll
-    for (int k = 0; k < N * N; ++k) a[k] = expf(a[k]);
+    for (int k = 0; k < N * N; ++k) a[k] = exp_shifted(a[k]);
     normalize_cols_n<N>(a);
     normalize_rows_n<N>(a);
 

@@ -23,6 +23,10 @@ cudaError_t launch_sinkhorn_bwd(const float* logits, const float* dP, float* dlo
 cudaError_t launch_implicit_bwd(const float* logits, const float* P, const float* dP, float* dlogits,
                                 int64_t n, cudaStream_t s);
 
+// y[i] = exp_shifted(x[i]): the exponential the projection kernels apply to
+// max-shifted logits.
+cudaError_t launch_exp_shifted(const float* x, float* y, int64_t n, cudaStream_t s);
+
 // n x n projection, n = 1..8 (n = 4 goes to the 4 x 4 kernels above).
 cudaError_t launch_birkhoff_fwd_n(const float* logits, float* P, int64_t n_mats, int n, bool newton, int iters,
                                   cudaStream_t s);

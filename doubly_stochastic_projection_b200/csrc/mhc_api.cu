@@ -143,6 +143,14 @@ int mhc_sinkhorn_bwd(const float* logits, const float* dP, float* dlogits, int64
     return cuda_status(mhc::launch_sinkhorn_bwd(logits, dP, dlogits, n_mats, it, static_cast<cudaStream_t>(stream)));
 }
 
+int mhc_exp_shifted(const float* x, float* y, int64_t n, void* stream)
+{
+    if (n < 0 || n > (int64_t(1) << 40)) return MHC_ERR_SIZE;
+    if (n == 0) return MHC_OK;
+    if (!x || !y) return MHC_ERR_NULL;
+    return cuda_status(mhc::launch_exp_shifted(x, y, n, static_cast<cudaStream_t>(stream)));
+}
+
 int mhc_residual_mix_fwd(const uint16_t* X, const float* H_res, const float* h_post, const uint16_t* F,
                          uint16_t* Y, int64_t T, int64_t C, void* stream)
 {

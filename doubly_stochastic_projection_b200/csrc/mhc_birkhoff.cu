@@ -113,6 +113,14 @@ Launch projection_launch(const void* kernel, int64_t n)
     return {kProjThreads, full};
 }
 
+__global__ void __launch_bounds__(kProjThreads) exp_shifted_kernel(const float* x, float* y, int64_t n)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) y[i] = exp_shifted(x[i]);
+}
+
 }  // namespace
 
 int device_sm_count()
@@ -182,6 +190,12 @@ cudaError_t launch_sinkhorn_bwd(const float* logits, const float* dP, float* dlo
 {
     const Launch L = projection_launch((const void*)sinkhorn_bwd_kernel, n);
     return launch_pdl(sinkhorn_bwd_kernel, L.grid, L.threads, 0, s, logits, dP, dlogits, n, iters);
+}
+
+cudaError_t launch_exp_shifted(const float* x, float* y, int64_t n, cudaStream_t s)
+{
+    const int grid = persistent_grid((const void*)exp_shifted_kernel, kProjThreads, 0, blocks_for(n, kProjThreads));
+    return launch_pdl(exp_shifted_kernel, grid, kProjThreads, 0, s, x, y, n);
 }
 
 }  // namespace mhc

@@ -171,6 +171,19 @@ MHC_API int mhc_birkhoff_bwd_n(const float *P, const float *dP, float *dlogits, 
                                void *stream);
 
 /*
+ * mhc_exp_shifted -- y[i] = e^{x[i]} as the projection kernels compute it for
+ * the max-shifted logits (x <= 0 there): the argument split of Cody and Waite
+ * (Software Manual for the Elementary Functions, 1980) around the hardware
+ * base-2 exponential, results below the smallest normal flushed to zero,
+ * x = -inf giving NaN.  Exposed so that its accuracy can be checked against a
+ * reference exponential; not needed to use the projection.
+ *
+ *   x, y  [n] float, device (4-byte alignment suffices); y may equal x.
+ *   n     >= 0, at most 2^40.
+ */
+MHC_API int mhc_exp_shifted(const float *x, float *y, int64_t n, void *stream);
+
+/*
  * mhc_sinkhorn_bwd -- backward of the MHC_SINKHORN forward with the same
  * `iters`: dlogits = dL/dlogits for upstream dP = dL/dP, the exact derivative
  * of the fixed-count iteration (the unrolled backward of the Sinkhorn baseline

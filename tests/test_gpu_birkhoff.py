@@ -164,11 +164,13 @@ def test_nonfinite_input_stays_in_its_matrix(orc):
     A = inputs.birkhoff_logits(64, "normal1", 71)
     A[5, 2, 1] = np.nan
     A[9, 0, 0] = np.inf
-    P = to_np64(api.birkhoff_fwd(to_gpu(A), "newton"))
-    bad = ~np.isfinite(P).all((1, 2))
-    assert bad[5] and bad[9] and bad.sum() == 2
-    ok = np.setdiff1d(np.arange(64), [5, 9])
-    assert np.abs(P[ok] - orc.newton(A[ok].astype(np.float64))).max() <= P_ABS_TOL
+    A[13, 3, 1] = -np.inf
+    for method in ("sinkhorn", "newton"):
+        P = to_np64(api.birkhoff_fwd(to_gpu(A), method))
+        bad = ~np.isfinite(P).all((1, 2))
+        assert bad[5] and bad[9] and bad[13] and bad.sum() == 3, method
+    ok = np.setdiff1d(np.arange(64), [5, 9, 13])
+    assert np.abs(P[ok] - orc.newton(A[ok].astype(np.float64))).max() <= P_ABS_TOL  # P: Newton's
 
 
 def test_degenerate_inputs(orc):
