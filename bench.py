@@ -63,8 +63,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-oracle sample budget")
     ap.add_argument("--profile", default=None,
-                    choices=["newton_fwd", "sinkhorn_fwd", "implicit_bwd", "mix_fwd", "mix_bwd",
-                             "proj_mix_fwd", "proj_mix_bwd"],
+                    choices=["newton_fwd", "sinkhorn_fwd", "sinkhorn_bwd", "implicit_bwd", "mix_fwd", "mix_bwd",
+                             "proj_mix_fwd", "proj_mix_bwd", "premap_fwd", "mix_post_bwd", "mix_premap_bwd"],
                     help="run one kernel --reps times on one case (for ncu) and exit")
     ap.add_argument("--size", type=int, default=1 << 22, help="--profile: matrices, or tokens T for the mix")
     ap.add_argument("--channels", type=int, default=4096, help="--profile: mix channels C")
@@ -590,7 +590,7 @@ def run_profile_case(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     k = args.profile
-    if k in ("newton_fwd", "sinkhorn_fwd", "implicit_bwd"):
+    if k in ("newton_fwd", "sinkhorn_fwd", "sinkhorn_bwd", "implicit_bwd"):
         n = args.size
         A = torch.from_numpy(inputs.birkhoff_logits(n, args.dist, 5)).to(dev)
         G = torch.from_numpy(inputs.upstream_grad(n, 6)).to(dev)
@@ -598,6 +598,7 @@ def run_profile_case(args):
         out = torch.empty_like(A)
         fn = {"newton_fwd": lambda: api.birkhoff_fwd(A, "newton", out=out),
               "sinkhorn_fwd": lambda: api.birkhoff_fwd(A, "sinkhorn", 20, out=out),
+              "sinkhorn_bwd": lambda: api.sinkhorn_bwd(G, A, 20),
               "implicit_bwd": lambda: api.birkhoff_bwd(G, P=P, out=out)}[k]
         desc = {"n_mats": n, "dist": args.dist}
     else:
@@ -607,10 +608,15 @@ def run_profile_case(args):
         h = torch.from_numpy(m["h_post"]).to(dev)
         H = api.birkhoff_fwd(lg, "newton")
         Y = torch.empty_like(X)
+        hpre = torch.from_numpy(inputs.h_post(args.size, 17)).to(dev) - 1.0
+        dx_in = dY[:, 0, :].contiguous()
         fn = {"mix_fwd": lambda: api.residual_mix_fwd(X, H, h, F, out=Y),
               "mix_bwd": lambda: api.residual_mix_bwd(X, H, h, F, dY, need_dlogits=True),
               "proj_mix_fwd": lambda: api.proj_mix_fwd(lg, h, X, F, out=Y, H_out=H),
-              "proj_mix_bwd": lambda: api.proj_mix_bwd(H, h, X, F, dY)}[k]
+              "proj_mix_bwd": lambda: api.proj_mix_bwd(H, h, X, F, dY),
+              "premap_fwd": lambda: api.premap_fwd(X, hpre),
+              "mix_post_bwd": lambda: api.mix_post_bwd(dY, F, h),
+              "mix_premap_bwd": lambda: api.mix_premap_bwd(X, H, hpre, dY, dx_in)}[k]
         desc = {"T": args.size, "C": args.channels}
     for _ in range(args.reps):
         fn()
