@@ -230,6 +230,22 @@ mix_premap_bwd_kernel(const uint4* X, const float* H, const float* hpre, const u
     ring.drain();
 }
 
+constexpr int kGainGroup = 4;
+
+// acc <- p acc (4 x 4, row-major)
+__device__ __forceinline__ void left_multiply(const float (&p)[16], float (&acc)[16])
+{
+    float nxt[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            nxt[4 * i + j] = fmaf(p[4 * i], acc[j], fmaf(p[4 * i + 1], acc[4 + j],
+                             fmaf(p[4 * i + 2], acc[8 + j], p[4 * i + 3] * acc[12 + j])));
+#pragma unroll
+    for (int k = 0; k < 16; ++k) acc[k] = nxt[k];
+}
+
 // Composite map across depth, one thread per token: M = P_{L-1} ... P_0.
 __global__ void __launch_bounds__(256)
 composite_gain_kernel(const float* P, float* M, float* gain_rows, float* gain_cols, int64_t L, int64_t T)
@@ -238,17 +254,20 @@ composite_gain_kernel(const float* P, float* M, float* gain_rows, float* gain_co
     for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < T; t += stride) {
         float acc[16];
         load16(P + 16 * t, acc);
-        for (int64_t l = 1; l < L; ++l) {
-            float p[16], nxt[16];
+        // layers in groups of kGainGroup: the group's loads are issued together,
+        // ahead of the serial chain of products
+        int64_t l = 1;
+        for (; l + kGainGroup <= L; l += kGainGroup) {
+            float p[kGainGroup][16];
+#pragma unroll
+            for (int g = 0; g < kGainGroup; ++g) load16(P + 16 * ((l + g) * T + t), p[g]);
+#pragma unroll
+            for (int g = 0; g < kGainGroup; ++g) left_multiply(p[g], acc);
+        }
+        for (; l < L; ++l) {
+            float p[16];
             load16(P + 16 * (l * T + t), p);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    nxt[4 * i + j] = fmaf(p[4 * i], acc[j], fmaf(p[4 * i + 1], acc[4 + j],
-                                     fmaf(p[4 * i + 2], acc[8 + j], p[4 * i + 3] * acc[12 + j])));
-#pragma unroll
-            for (int k = 0; k < 16; ++k) acc[k] = nxt[k];
+            left_multiply(p, acc);
         }
         float gr = 0.0f, gc = 0.0f;
 #pragma unroll

@@ -97,3 +97,15 @@ def test_composite_gain(orc):
             assert np.abs(to_np64(gr) - 1).max() <= 1e-4 and np.abs(to_np64(gc) - 1).max() <= 1e-4
         else:
             assert to_np64(gr).max() > 1.01   # finite Sinkhorn: the forward gain drifts
+
+
+@pytest.mark.parametrize("L", [1, 2, 4, 5, 7, 9])
+def test_composite_gain_layer_counts(orc, L):
+    # layer counts below, at and between multiples of the kernel's load group
+    T = 777
+    A = inputs.birkhoff_logits(L * T, "normal1", 91 + L)
+    P = api.birkhoff_fwd(to_gpu(A), "sinkhorn", 3).reshape(L, T, 4, 4).contiguous()
+    M, gr, gc = api.composite_gain(P)
+    rM, rgr, rgc = orc.composite_gain(to_np64(P))
+    assert np.abs(to_np64(M) - rM).max() <= 1e-5
+    assert np.abs(to_np64(gr) - rgr).max() <= 1e-5 and np.abs(to_np64(gc) - rgc).max() <= 1e-5
