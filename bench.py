@@ -538,6 +538,12 @@ def run_b200(args):
                 "frac": achieved / hbm, "traffic": traffic, "peak_source": hbm_src,
                 "algorithmic_bytes_per_launch": kbytes, "launch_us": kt * 1e6,
                 "note": "peak is the %s HBM copy bandwidth; the kernel is timed in isolation" % hbm_src}
+    if kname == "newton_fwd_kernel":
+        roofline["note"] += (". %d matrices are one wave of threads, so the launch lasts as long as its slowest "
+                             "warps (Newton iterations: max %d, per-warp maximum %.2f on average, mean %.2f): "
+                             "latency- and tail-bound, not bandwidth-bound; the large-batch fractions of the "
+                             "same kernel are in extras.sweep"
+                             % (N_MATS, newton_iters["max"], newton_iters["warp_max_mean"], newton_iters["mean"]))
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
