@@ -64,11 +64,13 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-oracle sample budget")
     ap.add_argument("--profile", default=None,
                     choices=["newton_fwd", "sinkhorn_fwd", "sinkhorn_bwd", "implicit_bwd", "mix_fwd", "mix_bwd",
-                             "proj_mix_fwd", "proj_mix_bwd", "premap_fwd", "mix_post_bwd", "mix_premap_bwd"],
+                             "proj_mix_fwd", "proj_mix_bwd", "premap_fwd", "mix_post_bwd", "mix_premap_bwd",
+                             "newton_fwd_n", "implicit_bwd_n"],
                     help="run one kernel --reps times on one case (for ncu) and exit")
     ap.add_argument("--size", type=int, default=1 << 22, help="--profile: matrices, or tokens T for the mix")
     ap.add_argument("--channels", type=int, default=4096, help="--profile: mix channels C")
     ap.add_argument("--dist", default="normal1", help="--profile: logit distribution")
+    ap.add_argument("--n", type=int, default=8, help="--profile newton_fwd_n / implicit_bwd_n: matrix size")
     ap.add_argument("--reps", type=int, default=3)
     return ap.parse_args()
 
@@ -425,6 +427,24 @@ def extras(dev, stream, flush, hbm, api, inputs):
         out["composite_gain"].append(row)
         del A
         torch.cuda.empty_cache()
+    # general n (other expansion rates): Newton forward and implicit backward
+    out["general_n"] = []
+    cnt = 1 << 20
+    for n in (2, 3, 6, 8):
+        A = torch.from_numpy(inputs.birkhoff_logits_n(cnt, n, 1.0, 20 + n)).to(dev)
+        G = torch.from_numpy(inputs.birkhoff_logits_n(cnt, n, 1.0, 120 + n)).to(dev)
+        P = torch.empty_like(A)
+        dl = torch.empty_like(A)
+        tf = event_time(lambda: api.birkhoff_fwd_n(A, "newton", out=P), reps, stream, flush)
+        api.birkhoff_fwd_n(A, "newton", out=P)
+        tb = event_time(lambda: api.birkhoff_bwd_n(G, P, out=dl), reps, stream, flush)
+        fb, bb = 8 * n * n * cnt, 12 * n * n * cnt
+        out["general_n"].append({
+            "n": n, "n_mats": cnt, "dist": "normal1",
+            "fwd_matrices_per_s": cnt / tf, "fwd_gbs": fb / tf / 1e9, "fwd_frac_hbm": fb / tf / 1e9 / hbm,
+            "bwd_matrices_per_s": cnt / tb, "bwd_gbs": bb / tb / 1e9, "bwd_frac_hbm": bb / tb / 1e9 / hbm})
+        del A, G, P, dl
+        torch.cuda.empty_cache()
     return out
 
 
@@ -596,7 +616,16 @@ def run_profile_case(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     k = args.profile
-    if k in ("newton_fwd", "sinkhorn_fwd", "sinkhorn_bwd", "implicit_bwd"):
+    if k in ("newton_fwd_n", "implicit_bwd_n"):
+        cnt = args.size
+        A = torch.from_numpy(inputs.birkhoff_logits_n(cnt, args.n, 1.0, 20 + args.n)).to(dev)
+        G = torch.from_numpy(inputs.birkhoff_logits_n(cnt, args.n, 1.0, 120 + args.n)).to(dev)
+        P = api.birkhoff_fwd_n(A, "newton")
+        out = torch.empty_like(A)
+        fn = {"newton_fwd_n": lambda: api.birkhoff_fwd_n(A, "newton", out=out),
+              "implicit_bwd_n": lambda: api.birkhoff_bwd_n(G, P, out=out)}[k]
+        desc = {"n_mats": cnt, "n": args.n}
+    elif k in ("newton_fwd", "sinkhorn_fwd", "sinkhorn_bwd", "implicit_bwd"):
         n = args.size
         A = torch.from_numpy(inputs.birkhoff_logits(n, args.dist, 5)).to(dev)
         G = torch.from_numpy(inputs.upstream_grad(n, 6)).to(dev)

@@ -117,6 +117,13 @@ def bf16_normal(shape, seed: int, device="cpu"):
     return out
 
 
+def birkhoff_logits_n(count: int, n: int, sigma: float, seed: int) -> np.ndarray:
+    """[count, n, n] float32 N(0, sigma^2) logits for the general-n projection
+    (also used as upstream gradients, sigma = 1)."""
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((int(count), int(n), int(n)), dtype=np.float32) * np.float32(sigma)).astype(np.float32)
+
+
 def birkhoff_workload(name: str):
     """(logits, dP) for the fixed-size projection workloads."""
     if name == "birkhoff_fwd_4096":

@@ -48,3 +48,11 @@ def test_mix_workload_small():
     assert m["X"].dtype == torch.bfloat16
     m2 = inputs.mix_workload("mix_T65536_C7168", T=6, C=32)
     assert torch.equal(m["X"], m2["X"]) and torch.equal(m["dY"], m2["dY"])
+
+
+def test_general_n_logits():
+    a = inputs.birkhoff_logits_n(1000, 6, 2.0, 5)
+    assert a.shape == (1000, 6, 6) and a.dtype == np.float32
+    assert np.array_equal(a, inputs.birkhoff_logits_n(1000, 6, 2.0, 5))
+    assert not np.array_equal(a, inputs.birkhoff_logits_n(1000, 6, 2.0, 6))
+    assert abs(a.std() - 2.0) < 0.05 and abs(a.mean()) < 0.05
