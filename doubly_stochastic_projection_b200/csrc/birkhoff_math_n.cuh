@@ -164,8 +164,11 @@ __device__ __forceinline__ int newton_project_n(float (&a)[N * N], int maxit)
 
         float W[N * (N - 1) / 2];
         float diag = 0.0f;
+        // (the outer bound j + 1 < N, not j < N: with an empty last pass the
+        // compiler stops unrolling this nest at N = 8 and moves a and W to
+        // local memory)
 #pragma unroll
-        for (int j = 0; j < N; ++j)
+        for (int j = 0; j + 1 < N; ++j)
 #pragma unroll
             for (int k = j + 1; k < N; ++k) {
                 float s = 0.0f;
@@ -251,12 +254,24 @@ __device__ __forceinline__ int newton_project_n(float (&a)[N * N], int maxit)
 // softmax Jacobian, lambda from the grounded-Laplacian solve, second pass.
 // Rows of P and of the upstream gradient are read from memory as they are
 // needed (twice each) rather than held, so that only the O(N^2 / 2) weights and
-// O(N) sums live in registers for the larger N.
-template <int N>
+// O(N) sums live in registers for the larger N.  P and Gin are read with plain
+// loads when they may be shared memory (kGlobal false) and through the
+// read-only cache otherwise; out may equal Gin, since row r of Gin is read
+// before row r of out is written and never after.
+template <int N, bool kGlobal>
+__device__ __forceinline__ float ld_in(const float* p)
+{
+    if constexpr (kGlobal)
+        return __ldg(p);
+    else
+        return *p;
+}
+
+template <int N, bool kGlobal = false>
 __device__ __forceinline__ void implicit_vjp_n(const float* P, const float* Gin, float* out)
 {
     if constexpr (N == 1) {
-        const float p = __ldg(P), g = __ldg(Gin);
+        const float p = ld_in<N, kGlobal>(P), g = ld_in<N, kGlobal>(Gin);
         out[0] = (p == p && g == g) ? 0.0f : __int_as_float(0x7fffffff);
     } else {
         double c[N], W[N * (N - 1) / 2];
@@ -268,8 +283,8 @@ __device__ __forceinline__ void implicit_vjp_n(const float* P, const float* Gin,
             float p[N], g[N];
 #pragma unroll
             for (int j = 0; j < N; ++j) {
-                p[j] = __ldg(P + N * r + j);
-                g[j] = __ldg(Gin + N * r + j);
+                p[j] = ld_in<N, kGlobal>(P + N * r + j);
+                g[j] = ld_in<N, kGlobal>(Gin + N * r + j);
             }
 #pragma unroll
             for (int k = 0; k + 1 < N; ++k) {
@@ -290,8 +305,8 @@ __device__ __forceinline__ void implicit_vjp_n(const float* P, const float* Gin,
             float p[N], g[N];
 #pragma unroll
             for (int j = 0; j < N; ++j) {
-                p[j] = __ldg(P + N * r + j);
-                g[j] = __ldg(Gin + N * r + j);
+                p[j] = ld_in<N, kGlobal>(P + N * r + j);
+                g[j] = ld_in<N, kGlobal>(Gin + N * r + j);
             }
 #pragma unroll
             for (int k = 0; k < N; ++k) {

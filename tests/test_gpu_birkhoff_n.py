@@ -5,7 +5,8 @@ import pytest
 import torch
 
 from doubly_stochastic_projection_b200 import api
-from _gpu_util import GRAD_REL_TOL, P_ABS_TOL, SUM_TOL, dev, per_matrix_rel_err, row_normalised, to_gpu, to_np64
+from _gpu_util import (GRAD_REL_TOL, P_ABS_TOL, SUM_TOL, dev, per_matrix_rel_err, row_normalised, sample_indices,
+                       to_gpu, to_np64)
 
 pytestmark = pytest.mark.gpu
 
@@ -62,3 +63,26 @@ def test_n_argument_errors():
     assert L.mhc_birkhoff_fwd_n(p, p, 4, 3, 2, 0, None) == 4   # refined is 4 x 4 only
     assert L.mhc_birkhoff_bwd_n(p, p, p, 4, 9, None) == 3
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("n", [5, 8])
+def test_projection_n_many_tiles_per_cta(orc, n):
+    # more matrices than one persistent grid holds (148 SMs x up to 5 CTAs x 128),
+    # so every CTA goes round its tile loop more than once, with a ragged last tile
+    count = 5 * 148 * 128 + 77
+    A = _logits(count, n, 1.0, 300 + n)
+    G = _logits(count, n, 1.0, 400 + n)
+    P_g = api.birkhoff_fwd_n(to_gpu(A), "newton")
+    P = to_np64(P_g)
+    assert np.isfinite(P).all() and P.min() >= 0
+    assert np.abs(P.sum(-1) - 1).max() <= SUM_TOL and np.abs(P.sum(-2) - 1).max() <= SUM_TOL
+    idx = sample_indices(count, 3000, 7 + n)
+    idx = np.concatenate([idx, np.arange(count - 77, count)])
+    ref = orc.newton(A[idx].astype(np.float64), tol=1e-12, max_iter=200)
+    assert np.abs(P[idx] - ref).max() <= P_ABS_TOL
+    S = to_np64(api.birkhoff_fwd_n(to_gpu(A), "sinkhorn", 20))
+    assert np.abs(S[idx] - orc.sinkhorn(A[idx].astype(np.float64), 20)).max() <= P_ABS_TOL
+    dl = to_np64(api.birkhoff_bwd_n(to_gpu(G), P_g))
+    dref = orc.implicit_bwd(row_normalised(P[idx]), G[idx].astype(np.float64))
+    rel, _ = per_matrix_rel_err(dl[idx].reshape(len(idx), -1), dref.reshape(len(idx), -1))
+    assert rel.max() <= GRAD_REL_TOL, rel.max()
