@@ -88,6 +88,9 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+E2E_CHUNKS = 4
+
+
 def csrc_hash():
     h = hashlib.sha256()
     d = os.path.join(ROOT, "doubly_stochastic_projection_b200", "csrc")
@@ -527,25 +530,64 @@ def run_b200(args):
     for _ in range(3):
         A_d.copy_(A_h, non_blocking=True)
     torch.cuda.synchronize()
+    # the batch goes through in E2E_CHUNKS pieces on three streams, so that the
+    # upload of a piece, the kernels of the previous one and the download of the
+    # one before overlap (PCIe carries both directions at once)
+    s_in = torch.cuda.Stream(dev)
+    s_out = torch.cuda.Stream(dev)
+    bounds = [N_MATS * c // E2E_CHUNKS for c in range(E2E_CHUNKS + 1)]
+
+    def pipelined_step(start):
+        s_in.wait_event(start)
+        for c in range(E2E_CHUNKS):
+            lo, hi = bounds[c], bounds[c + 1]
+            with torch.cuda.stream(s_in):
+                A_d[lo:hi].copy_(A_h[lo:hi], non_blocking=True)
+                G_d[lo:hi].copy_(G_h[lo:hi], non_blocking=True)
+                landed = torch.cuda.Event()
+                landed.record(s_in)
+            stream.wait_event(landed)
+            api.birkhoff_fwd(A_d[lo:hi], "newton", out=P[lo:hi])
+            api.birkhoff_bwd(G_d[lo:hi], P=P[lo:hi], out=dl[lo:hi])
+            computed = torch.cuda.Event()
+            computed.record(stream)
+            s_out.wait_event(computed)
+            with torch.cuda.stream(s_out):
+                P_h[lo:hi].copy_(P[lo:hi], non_blocking=True)
+                dl_h[lo:hi].copy_(dl[lo:hi], non_blocking=True)
+        fin = torch.cuda.Event()
+        fin.record(s_out)
+        stream.wait_event(fin)
+
     tot = 0.0
     for i in range(e2e_steps):
         flush()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        A_d.copy_(A_h, non_blocking=True)
-        G_d.copy_(G_h, non_blocking=True)
-        api.birkhoff_fwd(A_d, "newton", out=P)
-        api.birkhoff_bwd(G_d, P=P, out=dl)
-        P_h.copy_(P, non_blocking=True)
-        dl_h.copy_(dl, non_blocking=True)
+        pipelined_step(e0)
         e1.record(stream)
         e1.synchronize()
         tot += e0.elapsed_time(e1) * 1e-3
     t_e2e = max_over_ranks(tot / e2e_steps, pg, dev)
+    # one more step with the device inputs poisoned first: a kernel that read its
+    # inputs before their upload landed would leave NaN in the host results
+    A_d.fill_(float("nan"))
+    G_d.fill_(float("nan"))
+    P_h.zero_()
+    dl_h.zero_()
+    start = torch.cuda.Event()
+    start.record(stream)
+    pipelined_step(start)
+    torch.cuda.synchronize()
+    api.birkhoff_fwd(A, "newton", out=P)
+    api.birkhoff_bwd(G, P=P, out=dl)
+    matches = bool(torch.equal(dl_h, dl.cpu()) and torch.equal(P_h, P.cpu()))
     e2e = {"value": world * N_MATS / t_e2e, "unit": UNIT, "h2d_bytes_per_step": 2 * A.numel() * 4,
            "d2h_bytes_per_step": 2 * A.numel() * 4,
-           "path": "pinned host -> device copies, Newton fwd, implicit bwd, device -> host copies of P and dlogits"}
+           "path": "pinned host -> device copies, Newton fwd, implicit bwd, device -> host copies of P and "
+                   "dlogits, in %d pieces overlapped on three streams" % E2E_CHUNKS,
+           "matches_device_run": matches}
 
     # dominant kernel and its roofline (HBM-bound: algorithmic bytes / time)
     if t_fwd >= t_bwd:
