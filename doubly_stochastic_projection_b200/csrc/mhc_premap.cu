@@ -246,38 +246,66 @@ __device__ __forceinline__ void left_multiply(const float (&p)[16], float (&acc)
     for (int k = 0; k < 16; ++k) acc[k] = nxt[k];
 }
 
-// Composite map across depth, one thread per token: M = P_{L-1} ... P_0.
-__global__ void __launch_bounds__(256)
+// Composite map across depth: M = P_{L-1} ... P_0 per token.  One token per
+// thread would leave most of the GPU idle at the usual token counts (65536
+// threads for 65536 tokens), with each thread walking all L layers in turn;
+// so kGainSplit consecutive lanes share a token, each multiplying its own run
+// of about L / kGainSplit layers (kGainGroup loads ahead of the product
+// chain), and the partial products are combined in a shuffle tree,
+// M = Q_{S-1} ... Q_1 Q_0.
+constexpr int kGainThreads = 256;
+constexpr int kGainSplit = 4;
+constexpr int kGainTokensPerCta = kGainThreads / kGainSplit;
+
+__global__ void __launch_bounds__(kGainThreads)
 composite_gain_kernel(const float* P, float* M, float* gain_rows, float* gain_cols, int64_t L, int64_t T)
 {
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < T; t += stride) {
+    const int part = threadIdx.x % kGainSplit;
+    const int64_t lo = part * L / kGainSplit, hi = (part + 1) * L / kGainSplit;
+    // the loop bound depends on the CTA only, so every lane takes part in the shuffles
+    for (int64_t base = (int64_t)blockIdx.x * kGainTokensPerCta; base < T;
+         base += (int64_t)gridDim.x * kGainTokensPerCta) {
+        const int64_t t = base + threadIdx.x / kGainSplit;
+        const bool valid = t < T;
         float acc[16];
-        load16(P + 16 * t, acc);
-        // layers in groups of kGainGroup: the group's loads are issued together,
-        // ahead of the serial chain of products
-        int64_t l = 1;
-        for (; l + kGainGroup <= L; l += kGainGroup) {
-            float p[kGainGroup][16];
 #pragma unroll
-            for (int g = 0; g < kGainGroup; ++g) load16(P + 16 * ((l + g) * T + t), p[g]);
+        for (int k = 0; k < 16; ++k) acc[k] = (k % 5 == 0) ? 1.0f : 0.0f;  // identity
+        if (valid && lo < hi) {
+            load16(P + 16 * (lo * T + t), acc);
+            int64_t l = lo + 1;
+            for (; l + kGainGroup <= hi; l += kGainGroup) {
+                float p[kGainGroup][16];
 #pragma unroll
-            for (int g = 0; g < kGainGroup; ++g) left_multiply(p[g], acc);
-        }
-        for (; l < L; ++l) {
-            float p[16];
-            load16(P + 16 * (l * T + t), p);
-            left_multiply(p, acc);
-        }
-        float gr = 0.0f, gc = 0.0f;
+                for (int g = 0; g < kGainGroup; ++g) load16(P + 16 * ((l + g) * T + t), p[g]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            gr = fmaxf(gr, (fabsf(acc[4 * i]) + fabsf(acc[4 * i + 1])) + (fabsf(acc[4 * i + 2]) + fabsf(acc[4 * i + 3])));
-            gc = fmaxf(gc, (fabsf(acc[i]) + fabsf(acc[4 + i])) + (fabsf(acc[8 + i]) + fabsf(acc[12 + i])));
+                for (int g = 0; g < kGainGroup; ++g) left_multiply(p[g], acc);
+            }
+            for (; l < hi; ++l) {
+                float p[16];
+                load16(P + 16 * (l * T + t), p);
+                left_multiply(p, acc);
+            }
         }
-        if (M) store16(M + 16 * t, acc);
-        gain_rows[t] = gr;
-        gain_cols[t] = gc;
+        // combine the runs: lane part p (p a multiple of 2r) takes the run of
+        // lane p + r, which covers later layers, as the left factor
+#pragma unroll
+        for (int r = 1; r < kGainSplit; r <<= 1) {
+            float later[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) later[k] = __shfl_down_sync(0xffffffffu, acc[k], r);
+            if ((part & (2 * r - 1)) == 0) left_multiply(later, acc);
+        }
+        if (valid && part == 0) {
+            float gr = 0.0f, gc = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                gr = fmaxf(gr, (fabsf(acc[4 * i]) + fabsf(acc[4 * i + 1])) + (fabsf(acc[4 * i + 2]) + fabsf(acc[4 * i + 3])));
+                gc = fmaxf(gc, (fabsf(acc[i]) + fabsf(acc[4 + i])) + (fabsf(acc[8 + i]) + fabsf(acc[12 + i])));
+            }
+            if (M) store16(M + 16 * t, acc);
+            gain_rows[t] = gr;
+            gain_cols[t] = gc;
+        }
     }
 }
 
@@ -331,8 +359,9 @@ cudaError_t launch_mix_premap_bwd(const uint16_t* X, const float* H, const float
 cudaError_t launch_composite_gain(const float* P, float* M, float* gain_rows, float* gain_cols, int64_t L, int64_t T,
                                   cudaStream_t s)
 {
-    const int grid = persistent_grid((const void*)composite_gain_kernel, 256, 0, (T + 255) / 256);
-    composite_gain_kernel<<<grid, 256, 0, s>>>(P, M, gain_rows, gain_cols, L, T);
+    const int grid = persistent_grid((const void*)composite_gain_kernel, kGainThreads, 0,
+                                     (T + kGainTokensPerCta - 1) / kGainTokensPerCta);
+    composite_gain_kernel<<<grid, kGainThreads, 0, s>>>(P, M, gain_rows, gain_cols, L, T);
     return cudaGetLastError();
 }
 
