@@ -65,7 +65,7 @@ def parse():
     ap.add_argument("--profile", default=None,
                     choices=["newton_fwd", "sinkhorn_fwd", "sinkhorn_bwd", "implicit_bwd", "mix_fwd", "mix_bwd",
                              "proj_mix_fwd", "proj_mix_bwd", "premap_fwd", "mix_post_bwd", "mix_premap_bwd",
-                             "newton_fwd_n", "implicit_bwd_n"],
+                             "newton_fwd_n", "implicit_bwd_n", "composite_gain"],
                     help="run one kernel --reps times on one case (for ncu) and exit")
     ap.add_argument("--size", type=int, default=1 << 22, help="--profile: matrices, or tokens T for the mix")
     ap.add_argument("--channels", type=int, default=4096, help="--profile: mix channels C")
@@ -658,7 +658,13 @@ def run_profile_case(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     k = args.profile
-    if k in ("newton_fwd_n", "implicit_bwd_n"):
+    if k == "composite_gain":
+        L = 60
+        A = torch.from_numpy(inputs.birkhoff_logits(L * args.size, args.dist, 16)).to(dev)
+        P = api.birkhoff_fwd(A, "newton").reshape(L, args.size, 4, 4)
+        fn = lambda: api.composite_gain(P, need_M=False)
+        desc = {"layers": L, "tokens": args.size}
+    elif k in ("newton_fwd_n", "implicit_bwd_n"):
         cnt = args.size
         A = torch.from_numpy(inputs.birkhoff_logits_n(cnt, args.n, 1.0, 20 + args.n)).to(dev)
         G = torch.from_numpy(inputs.birkhoff_logits_n(cnt, args.n, 1.0, 120 + args.n)).to(dev)
