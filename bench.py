@@ -623,7 +623,9 @@ def run_b200(args):
     }
 
     line["clocks"] = clocks.summary()
-    if rank == 0 and not args.no_extras:
+    # the extras characterise one GPU; under torchrun the other ranks would sit in
+    # the closing barrier meanwhile, so they run only when there is one rank
+    if world == 1 and not args.no_extras:
         clocks.samples = []
         clocks.start()
         try:
