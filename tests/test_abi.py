@@ -71,3 +71,29 @@ def test_validation_rejects_before_any_cuda_call(L):
     assert L.mhc_birkhoff_fwd_n(fake, fake, 10, 9, 1, 0, None) == 3
     assert L.mhc_birkhoff_fwd_n(fake, fake, 10, 5, 2, 0, None) == 4
     assert L.mhc_birkhoff_fwd_n(None, None, 0, 5, 1, 0, None) == 0
+
+
+def test_validation_of_the_remaining_entry_points(L):
+    p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    fake = 1 << 20  # never dereferenced: every call below returns before launching
+    L.mhc_birkhoff_fwd_n.argtypes = [p, p, i64, i32, i32, i32, p]
+    L.mhc_birkhoff_bwd_n.argtypes = [p, p, p, i64, i32, p]
+    assert L.mhc_birkhoff_fwd_n(fake, fake, 10, 0, 1, 0, None) == 3
+    assert L.mhc_birkhoff_bwd_n(fake, fake, fake, 10, 9, None) == 3
+    assert L.mhc_birkhoff_bwd_n(fake, None, fake, 10, 3, None) == 1
+    L.mhc_composite_gain.argtypes = [p, p, p, p, i64, i64, p]
+    assert L.mhc_composite_gain(fake, None, fake, fake, 0, 10, None) == 3        # L >= 1
+    assert L.mhc_composite_gain(fake, None, fake, fake, 2, -1, None) == 3
+    assert L.mhc_composite_gain(fake, None, fake, fake, (1 << 20) + 1, 10, None) == 3
+    assert L.mhc_composite_gain(None, None, fake, fake, 2, 10, None) == 1
+    assert L.mhc_composite_gain(fake + 4, None, fake, fake, 2, 10, None) == 2
+    assert L.mhc_composite_gain(None, None, None, None, 2, 0, None) == 0       # no tokens
+    L.mhc_exp_shifted.argtypes = [p, p, i64, p]
+    assert L.mhc_exp_shifted(fake, fake, -1, None) == 3
+    assert L.mhc_exp_shifted(None, fake, 10, None) == 1
+    assert L.mhc_exp_shifted(None, None, 0, None) == 0
+    L.mhc_premap_bwd.argtypes = [p, p, p, p, p, i32, i64, i64, p]
+    assert L.mhc_premap_bwd(fake, fake, fake, fake, fake, 2, 4, 16, None) == 4     # accumulate is 0 or 1
+    L.mhc_residual_mix_bwd.argtypes = [p, p, p, p, p, p, p, p, p, p, i64, i64, p]
+    assert L.mhc_residual_mix_bwd(fake, fake, fake, fake, fake, fake, None, None, fake, None, 1 << 36, 1 << 24,
+                                  None) == 3                                    # T * 4 * C above 2^40
