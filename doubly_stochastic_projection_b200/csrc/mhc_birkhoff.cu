@@ -8,7 +8,9 @@
 // layout of the Birkhoff-acceleration summary (arXiv 2606.07574, §2.3) was
 // designed for an Ada GPU; here the projection is FP32/SFU-issue-bound
 // (Newton) or HBM-bound (backward), and a lane-per-entry layout would repeat
-// the 3x3 solve and the step logic on 16 lanes.
+// the 3x3 solve and the step logic on 16 lanes.  Every kernel here is
+// launched with programmatic dependent launch (pdl.cuh), so a forward and the
+// backward that follows it overlap their launch gap.
 #include <algorithm>
 #include <atomic>
 

@@ -11,9 +11,11 @@
 // The mix is a streaming, HBM-bound operation (about 1.1 fp32 FMA per byte
 // forward, 1.4 backward): there is no dense contraction to put on tensor
 // cores.  One CTA owns one token at a time; every thread moves whole 16-byte
-// vectors (8 bf16 channels) of each stream with streaming (evict-first)
-// loads and stores, so each warp touches 512 contiguous bytes per stream per
-// instruction.  The per-token H and h_post are broadcast loads.
+// vectors (8 bf16 channels) of each stream, so each warp touches 512
+// contiguous bytes per stream per instruction.  The forward uses streaming
+// (evict-first) loads and stores; the backward stages its nine input rows
+// through a per-thread cp.async ring in shared memory (see mix_bwd_kernel).
+// The per-token H and h_post are broadcast loads.
 #include "birkhoff_math.cuh"
 #include "launch.h"
 #include "mix_common.cuh"
