@@ -375,3 +375,43 @@ class BirkhoffProjection(torch.autograd.Function):
     def backward(ctx, dP):
         (P,) = ctx.saved_tensors
         return birkhoff_bwd(dP.contiguous(), P=P), None
+
+
+class ResidualMix(torch.autograd.Function):
+    """Autograd wrapper of the mix Y = H_res X + h_post (x) F (bf16 streams,
+    fp32 maps).  The backward is one mhc_residual_mix_bwd call; dH_res and
+    dh_post are computed only when an input needs them."""
+
+    @staticmethod
+    def forward(ctx, X, H_res, h_post, F):
+        X, H, h, F = X.contiguous(), H_res.contiguous(), h_post.contiguous(), F.contiguous()
+        Y = residual_mix_fwd(X, H, h, F)
+        ctx.save_for_backward(X, H, h, F)
+        return Y
+
+    @staticmethod
+    def backward(ctx, dY):
+        X, H, h, F = ctx.saved_tensors
+        o = residual_mix_bwd(X, H, h, F, dY.contiguous(), need_dH=ctx.needs_input_grad[1],
+                             need_dh_post=ctx.needs_input_grad[2])
+        return o["dX"], o["dH_res"], o["dh_post"], o["dF"]
+
+
+class ProjectedMix(torch.autograd.Function):
+    """Autograd wrapper of the fused path: logits -> H_res (Newton projection)
+    -> mix, forward in one kernel (mhc_proj_mix_fwd) and backward in one kernel
+    (mhc_proj_mix_bwd, the implicit backward chained in).  Saves H_res, not
+    the Newton iterates."""
+
+    @staticmethod
+    def forward(ctx, logits, h_post, X, F, iters: int = 0):
+        logits, h, X, F = logits.contiguous(), h_post.contiguous(), X.contiguous(), F.contiguous()
+        Y, H = proj_mix_fwd(logits, h, X, F, iters)
+        ctx.save_for_backward(H, h, X, F)
+        return Y
+
+    @staticmethod
+    def backward(ctx, dY):
+        H, h, X, F = ctx.saved_tensors
+        dX, dlogits, dh, dF = proj_mix_bwd(H, h, X, F, dY.contiguous())
+        return dlogits, dh, dX, dF, None
