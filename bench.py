@@ -241,9 +241,29 @@ def cpu_oracle_rate(seconds, n_sample=16384):
         el = time.perf_counter() - t0
         if el >= seconds:
             break
-    return {"value": done / el, "unit": UNIT, "cores": oracle.get_threads(), "kind": "oracle",
+    cores = oracle.get_threads()
+    # the same work on one core, on a quarter of the sample
+    quarter = len(A) // 4
+    A1 = np.concatenate([A[: quarter // 2], A[half: half + quarter // 2]])
+    G1 = np.concatenate([G[: quarter // 2], G[half: half + quarter // 2]])
+    oracle.set_threads(1)
+    try:
+        done1, t1 = 0, time.perf_counter()
+        while True:
+            P1 = oracle.newton(A1, tol=1e-10, max_iter=200)
+            oracle.implicit_bwd(P1, G1)
+            done1 += len(A1)
+            el1 = time.perf_counter() - t1
+            if el1 >= seconds / 4:
+                break
+    finally:
+        oracle.set_threads(cores)
+    return {"value": done / el, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": "%d matrices (%d of each half of the workload), Newton fwd to ||grad||<1e-10 + "
-                      "implicit bwd in fp64, repeated for %.1f s" % (len(A), half, el)}
+                      "implicit bwd in fp64, repeated for %.1f s" % (len(A), half, el),
+            "single_core": {"value": done1 / el1, "unit": UNIT, "cores": 1,
+                            "sample": "%d matrices (%d of each half), the same work, repeated for %.1f s"
+                                      % (len(A1), len(A1) // 2, el1)}}
 
 
 def run_reference(args):
