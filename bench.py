@@ -450,10 +450,11 @@ def extras(dev, stream, flush, hbm, api, inputs):
         out["composite_gain"].append(row)
         del A
         torch.cuda.empty_cache()
-    # general n (other expansion rates): Newton forward and implicit backward
+    # general n (other expansion rates): Newton forward and implicit backward,
+    # each n on about 256 MB of logits so that launch overhead does not dominate
     out["general_n"] = []
-    cnt = 1 << 20
     for n in (2, 3, 6, 8):
+        cnt = (1 << 26) // (n * n)
         A = torch.from_numpy(inputs.birkhoff_logits_n(cnt, n, 1.0, 20 + n)).to(dev)
         G = torch.from_numpy(inputs.birkhoff_logits_n(cnt, n, 1.0, 120 + n)).to(dev)
         P = torch.empty_like(A)
