@@ -97,3 +97,25 @@ def test_validation_of_the_remaining_entry_points(L):
     L.mhc_residual_mix_bwd.argtypes = [p, p, p, p, p, p, p, p, p, p, i64, i64, p]
     assert L.mhc_residual_mix_bwd(fake, fake, fake, fake, fake, fake, None, None, fake, None, 1 << 36, 1 << 24,
                                   None) == 3                                    # T * 4 * C above 2^40
+
+
+def test_header_is_plain_c(tmp_path):
+    # the boundary is usable from C: the header compiles as strict C99 and a C
+    # program links the library and runs a host-only call
+    import shutil
+    import subprocess
+
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "t.c"
+    src.write_text('#include <stdio.h>\n#include "mhc_birkhoff.h"\n'
+                   "int main(void) {\n"
+                   "    if (mhc_version() < 100) return 2;\n"
+                   "    return mhc_birkhoff_fwd(NULL, NULL, -1, MHC_NEWTON, 0, NULL) == MHC_ERR_SIZE ? 0 : 1;\n"
+                   "}\n")
+    inc = os.path.join(build.ROOT, "include")
+    libdir = os.path.dirname(build.LIB_PATH)
+    exe = tmp_path / "t"
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", inc, str(src),
+                           "-L", libdir, "-lmhc_b200", "-Wl,-rpath," + libdir, "-o", str(exe)])
+    assert subprocess.call([str(exe)]) == 0
