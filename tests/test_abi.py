@@ -119,3 +119,13 @@ def test_header_is_plain_c(tmp_path):
     subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", inc, str(src),
                            "-L", libdir, "-lmhc_b200", "-Wl,-rpath," + libdir, "-o", str(exe)])
     assert subprocess.call([str(exe)]) == 0
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path, monkeypatch):
+    # no CPU or torch fallback: a missing library is an error, not a slow path
+    from doubly_stochastic_projection_b200 import api
+
+    monkeypatch.setattr(api, "_lib", None)
+    monkeypatch.setattr(api._build, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError, match="no fallback"):
+        api.lib()
