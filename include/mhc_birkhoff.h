@@ -101,7 +101,7 @@ enum mhc_method {
  *             ([BA] §2) -- found by Newton's method on the dual reduced to the
  *             three column potentials g_0..g_2 (g_3 = 0) with closed-form
  *             gradient (column sums minus one) and Hessian ([BA] §2.1).
- *             `iters` is the maximum Newton iteration count; 0 selects 50.
+ *             `iters` is the maximum Newton iteration count; 0 selects 100.
  *             Tolerance: every column sum within 1e-6 of one (rows are exact
  *             to rounding by construction), so every entry of P is accurate
  *             to about 1e-6 in absolute terms.
@@ -239,7 +239,7 @@ MHC_API int mhc_residual_mix_bwd(const uint16_t *X, const float *H_res, const fl
 /*
  * mhc_proj_mix_fwd -- fused projection + mix: H_res = Newton projection of
  * logits (written out for the backward), then Y = H_res . X + h_post (x) F,
- * in one kernel.  `iters` as for MHC_NEWTON (0 selects 50).
+ * in one kernel.  `iters` as for MHC_NEWTON (0 selects 100).
  *
  *   logits [T][4][4] float, read.    H_res [T][4][4] float, written.
  *   Other arguments as mhc_residual_mix_fwd.
