@@ -10,19 +10,23 @@ shard of matrices; the projection is independent per matrix, so no collective
 runs on the data path).
 
 Timing: W untimed warm-up steps; then, between a barrier and a device
-synchronisation on both sides, exactly K steps, each bracketed by CUDA events
-recorded on the stream the kernels run on, with the L2 cache flushed (a 512 MiB
-read) before every step and outside its events, because the step's 32 MiB
-working set would otherwise stay in the 126 MB L2.  The reported time is the
-sum of the K step durations, maximised over ranks.
+synchronisation on both sides, exactly K steps run back to back -- captured
+once in a CUDA graph and replayed between two CUDA events recorded on the
+launching stream -- so that no host launch gap, event or cache flush sits
+between the steps.  The inputs are larger than L2: the steps rotate over 16
+replicas of the batch's inputs and outputs (512 MiB in all, four times the
+126 MB L2), so every step reads inputs last touched 15 steps earlier and
+evicted since.  The reported time is the K-step interval, maximised over
+ranks.
 
-Also reported: the end-to-end figure through the public API with host buffers
-(pinned host -> device copies of the inputs and device -> host copies of the
-outputs inside the timed region), the roofline of the dominant kernel against
-the measured HBM copy bandwidth, the fp64 CPU oracle timed on the host cores,
-SM clocks sampled through NVML during the timed region, and (unless
---no-extras) the 1M/4M/16M sweep, 20-iteration Sinkhorn, and the residual-mix
-workloads.
+Also reported: the end-to-end figure through the C ABI with pinned host buffers
+(mhc_birkhoff_fwd_bwd_host: host -> device copies, kernels, device -> host
+copies, pipelined, inside the timed region), the roofline of the dominant kernel
+against the measured HBM copy bandwidth and the FP32 and MUFU issue peaks, the
+fp64 CPU oracle timed on the host cores, SM clocks through NVML, and (unless
+--no-extras) the 1M/4M/16M sweep, 20-iteration Sinkhorn, the layouts of the
+Newton forward, and the residual-mix workloads.  The last key of the JSON line
+is a compact ``targets`` summary of the fractions the extras measured.
 
 ``--impl reference`` times the fp64 CPU oracle (the reference implementation
 of what the kernels compute) on bounded samples of the same workload.
@@ -49,8 +53,23 @@ WORKLOAD = "birkhoff_fwd_bwd_131072"
 N_MATS = 131072
 BYTES_FWD = 128   # logits in, P out
 BYTES_BWD = 192   # P and dP in, dlogits out
+REPLICAS = 16     # rotating copies of the step's working set (16 x 32 MiB)
 L2_FLUSH_BYTES = 512 << 20
 FALLBACK_HBM_GBS = 6650.0
+SM_COUNT = 148
+FP32_LANES_PER_SM = 128   # FP32 lane operations per SM per clock
+MUFU_LANES_PER_SM = 16    # SFU (MUFU) lane operations per SM per clock
+
+# Algorithmic work of the Newton forward per matrix, counted from its
+# arithmetic (FP32 add / multiply / fma lane operations, and MUFU operations:
+# reciprocals and base-2 exponentials).  Start-up: two max shifts, 16
+# compensated exponentials, one Sinkhorn round.  One iteration: column sums
+# and error, the six Laplacian weights, damping, the grounded-Laplacian
+# solve, three column factors, four row sums and the multiplicative update.
+# The near-permutation step repeats an iteration's work on a cancellation-free
+# gradient.  Line-search trials are not counted.
+NEWTON_OPS = {"fp32_start": 168, "mufu_start": 24, "fp32_iter": 120, "mufu_iter": 10,
+              "fp32_polish": 136, "mufu_polish": 10}
 
 
 def parse():
@@ -61,18 +80,30 @@ def parse():
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--no-extras", action="store_true", help="skip the sweep and mix extras")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-oracle sample budget")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-oracle sample budget (Newton leg)")
+    ap.add_argument("--e2e-pieces", type=int, default=8, help="pieces of the end-to-end host pipeline")
     ap.add_argument("--profile", default=None,
                     choices=["newton_fwd", "sinkhorn_fwd", "sinkhorn_bwd", "implicit_bwd", "mix_fwd", "mix_bwd",
                              "proj_mix_fwd", "proj_mix_bwd", "premap_fwd", "mix_post_bwd", "mix_premap_bwd",
                              "newton_fwd_n", "implicit_bwd_n", "composite_gain"],
                     help="run one kernel --reps times on one case (for ncu) and exit")
+    ap.add_argument("--method", default="newton", help="--profile newton_fwd: projection method")
     ap.add_argument("--size", type=int, default=1 << 22, help="--profile: matrices, or tokens T for the mix")
     ap.add_argument("--channels", type=int, default=4096, help="--profile: mix channels C")
     ap.add_argument("--dist", default="normal1", help="--profile: logit distribution")
     ap.add_argument("--n", type=int, default=8, help="--profile newton_fwd_n / implicit_bwd_n: matrix size")
     ap.add_argument("--reps", type=int, default=3)
     return ap.parse_args()
+
+
+def headline_config(world):
+    """The workload description both arms print."""
+    return {"workload": WORKLOAD, "n_mats_per_gpu": N_MATS,
+            "logits": "first half N(0,1), second half N(0,10^2), seed 2 (+7919*rank)",
+            "step": "Newton fwd (to max|colsum-1|<1e-6, near-permutation relative-accuracy step) + implicit bwd",
+            "l2": "inputs larger than L2: the steps rotate over %d replicas of the batch's inputs and outputs "
+                  "(%d MiB, 4x the L2)" % (REPLICAS, REPLICAS * 32),
+            "parallelism": "token-sharded replicas, no collective" if world > 1 else "single GPU"}
 
 
 # ----------------------------------------------------------------- helpers
@@ -86,9 +117,6 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
-
-
-E2E_CHUNKS = 4
 
 
 def csrc_hash():
@@ -124,7 +152,7 @@ class ClockSampler:
         0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, index, period=0.01):
+    def __init__(self, index, period=0.002):
         self.samples = []
         self.period = period
         self._stop = threading.Event()
@@ -165,10 +193,10 @@ class ClockSampler:
     def stop(self):
         self._stop.set()
 
-    def summary(self):
+    def summary(self, samples=None):
         if not self.ok:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": "unavailable"}
-        s = list(self.samples)
+        s = list(self.samples if samples is None else samples)
         mhz = [m for m, _ in s]
         mask = 0
         for _, r in s:
@@ -219,9 +247,20 @@ def barrier(pg, device):
 # ----------------------------------------------------------------- CPU oracle
 
 
+def _timed_loop(fn, seconds):
+    done, t0 = 0, time.perf_counter()
+    while True:
+        done += fn()
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            return done, el
+
+
 def cpu_oracle_rate(seconds, n_sample=16384):
-    """fp64 oracle Newton forward + implicit backward on a bounded sample of the
-    workload (matrices of both halves), repeated for about `seconds`."""
+    """The fp64 oracle, as it stands, on bounded samples of the benchmark's
+    workloads: the headline Newton fwd + implicit bwd (matrices/s), the
+    20-round Sinkhorn forward (matrices/s) and the residual mix forward and
+    backward of both mix workloads (tokens/s); all host cores, and one core."""
     import numpy as np
 
     import oracle
@@ -233,29 +272,33 @@ def cpu_oracle_rate(seconds, n_sample=16384):
     A = A[idx].astype(np.float64)
     G = G[idx].astype(np.float64)
     oracle.newton(A[:64])
-    done, t0 = 0, time.perf_counter()
-    while True:
-        P = oracle.newton(A, tol=1e-10, max_iter=200)
-        oracle.implicit_bwd(P, G)
-        done += len(A)
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
     cores = oracle.get_threads()
-    # the same work on one core, on a quarter of the sample
+
+    def newton_step(a, g):
+        P = oracle.newton(a, tol=1e-10, max_iter=200)
+        oracle.implicit_bwd(P, g)
+        return len(a)
+
+    done, el = _timed_loop(lambda: newton_step(A, G), seconds)
     quarter = len(A) // 4
     A1 = np.concatenate([A[: quarter // 2], A[half: half + quarter // 2]])
     G1 = np.concatenate([G[: quarter // 2], G[half: half + quarter // 2]])
+    sk_done, sk_el = _timed_loop(lambda: (oracle.sinkhorn(A, 20), len(A))[1], seconds / 4)
+    mix = {}
+    for name, T in (("mix_T16384_C4096", 256), ("mix_T65536_C7168", 128)):
+        m = inputs.mix_workload(name, device="cpu", T=T)
+        bits = lambda t: t.contiguous().view(__import__("torch").int16).numpy().view(np.uint16)
+        X, F, dY = bits(m["X"]), bits(m["F"]), bits(m["dY"])
+        H = oracle.newton(m["logits"].astype(np.float64))
+        hp = m["h_post"].astype(np.float64)
+        f_done, f_el = _timed_loop(lambda: (oracle.mix_fwd(X, H, hp, F), T)[1], seconds / 8)
+        b_done, b_el = _timed_loop(lambda: (oracle.mix_bwd(X, H, hp, F, dY), T)[1], seconds / 8)
+        mix[name] = {"fwd_tokens_per_s": f_done / f_el, "bwd_tokens_per_s": b_done / b_el,
+                     "sample": "%d tokens (C = %d), fp64 over bf16-decoded inputs" % (T, m["C"])}
     oracle.set_threads(1)
     try:
-        done1, t1 = 0, time.perf_counter()
-        while True:
-            P1 = oracle.newton(A1, tol=1e-10, max_iter=200)
-            oracle.implicit_bwd(P1, G1)
-            done1 += len(A1)
-            el1 = time.perf_counter() - t1
-            if el1 >= seconds / 4:
-                break
+        done1, el1 = _timed_loop(lambda: newton_step(A1, G1), seconds / 4)
+        sk1, skel1 = _timed_loop(lambda: (oracle.sinkhorn(A1, 20), len(A1))[1], seconds / 8)
     finally:
         oracle.set_threads(cores)
     return {"value": done / el, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -263,7 +306,11 @@ def cpu_oracle_rate(seconds, n_sample=16384):
                       "implicit bwd in fp64, repeated for %.1f s" % (len(A), half, el),
             "single_core": {"value": done1 / el1, "unit": UNIT, "cores": 1,
                             "sample": "%d matrices (%d of each half), the same work, repeated for %.1f s"
-                                      % (len(A1), len(A1) // 2, el1)}}
+                                      % (len(A1), len(A1) // 2, el1)},
+            "sinkhorn20_fwd": {"value": sk_done / sk_el, "unit": UNIT, "cores": cores,
+                               "single_core": sk1 / skel1,
+                               "sample": "the same %d matrices, 20 Sinkhorn-Knopp rounds in fp64" % len(A)},
+            "mix": {"unit": "tokens/s", "cores": cores, **mix}}
 
 
 def run_reference(args):
@@ -283,7 +330,6 @@ def run_reference(args):
     # take about a minute at most
     total_budget = 60.0
     per_step = max(64, min(N_MATS, int(2.0e6 * total_budget / max(1, args.steps + args.warmup))))
-    rng = np.random.default_rng(0)
 
     def step(i):
         s = (i * per_step) % (N_MATS - per_step + 1)
@@ -301,18 +347,18 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "n_mats": N_MATS, "matrices_per_step_sample": per_step,
-                   "path": "Newton fwd + implicit bwd", "l2": "host"},
+        "config": headline_config(world),
         "cpu_baseline": {"kind": "oracle", "cores": oracle.get_threads(), "value": value, "unit": UNIT,
-                         "sample": "%d consecutive matrices of the workload per step, fp64 Newton fwd + "
-                                   "implicit bwd" % per_step},
+                         "sample": "%d consecutive matrices of the %d-matrix workload per step (the first rank's "
+                                   "shard), fp64 Newton fwd to ||grad||<1e-10 + implicit bwd, on the host cores"
+                                   % (per_step, N_MATS)},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
-# ----------------------------------------------------------------- GPU arm
+# ----------------------------------------------------------------- GPU timing
 
 
 def event_time(fn, reps, stream, flush=None):
@@ -335,8 +381,94 @@ def event_time(fn, reps, stream, flush=None):
     return tot / reps
 
 
-def extras(dev, stream, flush, hbm, api, inputs):
-    import numpy as np
+def capture(launches):
+    """A CUDA graph of the given callables, launched in order (each enqueues
+    work on the current stream)."""
+    import torch
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for f in launches:
+            f()
+    return g
+
+
+def upload(g, stream):
+    """Uploads an instantiated graph to the device ahead of its first launch
+    (cuGraphUpload), so that the first replay does not pay for it."""
+    import ctypes
+
+    import torch
+
+    try:
+        cu = ctypes.CDLL("libcuda.so.1")
+        cu.cuGraphUpload.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+        rc = cu.cuGraphUpload(ctypes.c_void_p(int(g.raw_cuda_graph_exec())), ctypes.c_void_p(stream.cuda_stream))
+        torch.cuda.synchronize()
+        return rc == 0
+    except Exception:
+        return False
+
+
+def graph_time(g, stream, count):
+    """Device time (s) of one replay of graph g, per unit of `count`."""
+    import torch
+
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) * 1e-3 / count
+
+
+def backtoback_time(make, n_rep, launches, stream):
+    """Per-launch device time (s) of `launches` back-to-back launches, launch i
+    working on replica i % n_rep (make(r) returns replica r's launcher), as
+    one CUDA graph replayed once untimed and once timed."""
+    reps = [make(r) for r in range(n_rep)]
+    g = capture([reps[i % n_rep] for i in range(launches)])
+    graph_time(g, stream, launches)
+    t = graph_time(g, stream, launches)
+    del g
+    return t
+
+
+# ----------------------------------------------------------------- rooflines
+
+
+def projection_roofline(kname, n, t, hbm, mhz, its_mean=None, polished=None):
+    """The three roofs of a projection launch of n matrices taking t seconds:
+    HBM (algorithmic bytes), FP32 lane operations and MUFU operations (the
+    method's executed work at the measured mean iteration count).  The bound
+    is the roof with the longest minimum time."""
+    f = (mhz or 1965) * 1e6
+    fp32_peak = SM_COUNT * FP32_LANES_PER_SM * f
+    mufu_peak = SM_COUNT * MUFU_LANES_PER_SM * f
+    roofs = {}
+    nbytes = (BYTES_FWD if "fwd" in kname else BYTES_BWD) * n
+    roofs["hbm"] = {"min_us": nbytes / (hbm * 1e9) * 1e6, "achieved": nbytes / t / 1e9, "peak": hbm,
+                    "unit": "GB/s", "work_per_launch": nbytes}
+    if its_mean is not None:
+        o = NEWTON_OPS
+        fp = n * (o["fp32_start"] + o["fp32_iter"] * its_mean + o["fp32_polish"] * polished)
+        mu = n * (o["mufu_start"] + o["mufu_iter"] * its_mean + o["mufu_polish"] * polished)
+        roofs["fp32"] = {"min_us": fp / fp32_peak * 1e6, "achieved": fp / t / 1e12, "peak": fp32_peak / 1e12,
+                         "unit": "T lane-ops/s", "work_per_launch": fp}
+        roofs["mufu"] = {"min_us": mu / mufu_peak * 1e6, "achieved": mu / t / 1e12, "peak": mufu_peak / 1e12,
+                         "unit": "T ops/s", "work_per_launch": mu}
+    for r in roofs.values():
+        r["frac"] = r["achieved"] / r["peak"]
+    bound = max(roofs, key=lambda k: roofs[k]["min_us"])
+    return bound, roofs
+
+
+# ----------------------------------------------------------------- extras
+
+
+def extras(dev, stream, flush, hbm, mhz, api, inputs):
     import torch
 
     out = {"sweep": [], "sinkhorn20": [], "mix": []}
@@ -349,18 +481,24 @@ def extras(dev, stream, flush, hbm, api, inputs):
             dl = torch.empty_like(A)
             api.birkhoff_fwd(A, "newton", out=P)
             _, its = api.birkhoff_fwd_diag(A)
+            pol = near_permutation_fraction(P)
             tf = event_time(lambda: api.birkhoff_fwd(A, "newton", out=P), reps, stream, flush)
-            tr = event_time(lambda: api.birkhoff_fwd(A, "newton_refined", out=dl), reps, stream, flush)
+            ta = event_time(lambda: api.birkhoff_fwd(A, "newton_absolute", out=dl), reps, stream, flush)
             tb = event_time(lambda: api.birkhoff_bwd(G, P=P, out=dl), reps, stream, flush)
             itn = its.float()
+            its_mean = float(itn.mean())
+            bound, roofs = projection_roofline("newton_fwd", n, tf, hbm, mhz, its_mean, pol)
             out["sweep"].append({
                 "n_mats": n, "dist": dist,
                 "fwd_matrices_per_s": n / tf, "bwd_matrices_per_s": n / tb, "fwd_bwd_matrices_per_s": n / (tf + tb),
                 "fwd_gbs": BYTES_FWD * n / tf / 1e9, "bwd_gbs": BYTES_BWD * n / tb / 1e9,
                 "fwd_frac_hbm": BYTES_FWD * n / tf / 1e9 / hbm, "bwd_frac_hbm": BYTES_BWD * n / tb / 1e9 / hbm,
                 "fwd_bwd_frac_hbm": (BYTES_FWD + BYTES_BWD) * n / (tf + tb) / 1e9 / hbm,
-                "fwd_refined_matrices_per_s": n / tr, "fwd_refined_frac_hbm": BYTES_FWD * n / tr / 1e9 / hbm,
-                "newton_iters_mean": float(itn.mean()), "newton_iters_max": int(its.max()),
+                "fwd_frac_fp32": roofs["fp32"]["frac"], "fwd_bound": bound,
+                "fwd_frac_of_bound": roofs[bound]["frac"],
+                "fwd_absolute_matrices_per_s": n / ta, "fwd_absolute_frac_hbm": BYTES_FWD * n / ta / 1e9 / hbm,
+                "near_permutation_step_fraction": pol,
+                "newton_iters_mean": its_mean, "newton_iters_max": int(its.max()),
                 "newton_iters_warp_max_mean": float(itn.reshape(-1, 32).max(1).values.mean()),
             })
             if dist in ("normal1", "normal10"):
@@ -421,6 +559,7 @@ def extras(dev, stream, flush, hbm, api, inputs):
         tp = event_time(lambda: api.premap_fwd(X, hpre, out=x_in), reps, stream, flush)
         t_split = event_time(lambda: (api.mix_post_bwd(dY, F, h),
                                       api.mix_premap_bwd(X, H, hpre, dY, dx_in, need_dlogits=True)), reps, stream, flush)
+
         def unsplit():
             o = api.residual_mix_bwd(X, H, h, F, dY, need_dlogits=True)
             api.premap_bwd(X, hpre, dx_in, dX=o["dX"], accumulate=True)
@@ -472,8 +611,50 @@ def extras(dev, stream, flush, hbm, api, inputs):
     return out
 
 
+def near_permutation_fraction(P):
+    """Fraction of matrices that take the near-permutation step (every row
+    maximum above 0.6 and some row maximum above 0.98), from the output."""
+    m = P.max(-1).values
+    return float(((m.min(-1).values > 0.6) & (m.max(-1).values > 0.98)).float().mean())
+
+
+def targets_summary(line, hbm):
+    """The fractions the benchmark spec's targets are stated in, compactly, for the
+    tail of the JSON line."""
+    ex = line.get("extras") or {}
+    t = {"hbm_peak_gbs": hbm}
+    size_name = {1 << 20: "1M", 1 << 22: "4M", 1 << 24: "16M"}
+    short = {"normal1": "n1", "normal3": "n3", "normal10": "n10", "near_identity": "nid", "near_permutation": "nperm"}
+    fwd, fb, bound = {}, {}, {}
+    for r in ex.get("sweep", []):
+        k = "%s_%s" % (size_name.get(r["n_mats"], r["n_mats"]), short.get(r["dist"], r["dist"]))
+        fwd[k] = round(r["fwd_frac_hbm"], 3)
+        fb[k] = round(r["fwd_bwd_frac_hbm"], 3)
+        bound[k] = "%s %.3f" % (r["fwd_bound"], r["fwd_frac_of_bound"])
+    if fwd:
+        t["newton_fwd_frac_hbm"] = fwd
+        t["newton_fwd_frac_of_its_bound"] = bound
+        t["newton_fwd_bwd_frac_hbm"] = fb
+    sk = {"%s_%s" % (size_name.get(r["n_mats"], r["n_mats"]), short[r["dist"]]): round(r["fwd_frac_hbm"], 3)
+          for r in ex.get("sinkhorn20", [])}
+    if sk:
+        t["sinkhorn20_fwd_frac_hbm"] = sk
+    for r in ex.get("mix", []):
+        t[r["workload"]] = {"fwd": round(r["fwd_frac_hbm"], 3), "bwd": round(r["bwd_frac_hbm"], 3),
+                            "fused_fwd": round(r["fused_fwd_frac_hbm"], 3),
+                            "fused_bwd": round(r["fused_bwd_frac_hbm"], 3),
+                            "fused_fwd_bwd_tokens_per_s": round(r["fused_fwd_bwd_tokens_per_s"])}
+    rl = line.get("roofline", {})
+    t["headline"] = {"matrices_per_s": round(line["value"]), "e2e_matrices_per_s": round(line["e2e"]["value"]),
+                     "dominant_kernel": rl.get("kernel"), "bound": rl.get("bound"),
+                     "frac": round(rl.get("frac", 0.0), 3)}
+    return t
+
+
+# ----------------------------------------------------------------- GPU arm
+
+
 def run_b200(args):
-    import numpy as np
     import torch
 
     from doubly_stochastic_projection_b200 import api, inputs
@@ -492,166 +673,179 @@ def run_b200(args):
         G_np = inputs.upstream_grad(N_MATS, 102 + 7919 * rank)
     A = torch.from_numpy(A_np).to(dev)
     G = torch.from_numpy(G_np).to(dev)
-    P = torch.empty_like(A)
-    dl = torch.empty_like(A)
-    flush_buf = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    # R replicas of inputs and outputs; step i works on replica i % R
+    As = [A.clone() for _ in range(REPLICAS)]
+    Gs = [G.clone() for _ in range(REPLICAS)]
+    Ps = [torch.empty_like(A) for _ in range(REPLICAS)]
+    dls = [torch.empty_like(A) for _ in range(REPLICAS)]
+    P, dl = Ps[0], dls[0]
 
-    def flush():
-        # a read of 4x the L2 size: evicts the previous step's lines and leaves
-        # L2 holding clean lines only, so no write-back of earlier data lands
-        # inside the next step's events
-        flush_buf.sum()
+    def step_on(r):
+        def f():
+            api.birkhoff_fwd(As[r], "newton", out=Ps[r])
+            api.birkhoff_bwd(Gs[r], P=Ps[r], out=dls[r])
+        return f
 
-    def step():
-        api.birkhoff_fwd(A, "newton", out=P)
-        api.birkhoff_bwd(G, P=P, out=dl)
-
-    for _ in range(max(3, args.warmup)):
-        flush()
-        step()
+    steps = [step_on(r) for r in range(REPLICAS)]
+    K, W = args.steps, max(3, args.warmup)
+    for i in range(W):
+        steps[i % REPLICAS]()
     torch.cuda.synchronize()
+    timed = capture([steps[(W + i) % REPLICAS] for i in range(K)])
+    uploaded = upload(timed, stream)
 
     clocks = ClockSampler(local)
-    K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
     barrier(pg, dev)
     torch.cuda.synchronize()
     clocks.start()
-    for i in range(K):
-        flush()
-        e0, e1 = ev[i]
-        e0.record(stream)
-        step()
-        e1.record(stream)
+    e0.record(stream)
+    timed.replay()
+    e1.record(stream)
     torch.cuda.synchronize()
     clocks.pause()
     barrier(pg, dev)
-    t_step = sum(e0.elapsed_time(e1) for e0, e1 in ev) * 1e-3
+    t_step = e0.elapsed_time(e1) * 1e-3
     t_max = max_over_ranks(t_step, pg, dev)
     value = world * N_MATS * K / t_max
     gpu_launches = 2 * K
-    # per-kernel split, timed separately (an event between the two kernels
-    # would itself serialise the second launch behind the first)
-    t_fwd = event_time(lambda: api.birkhoff_fwd(A, "newton", out=P), 50, stream, flush) * K
-    t_bwd = event_time(lambda: api.birkhoff_bwd(G, P=P, out=dl), 50, stream, flush) * K
+    in_region = list(clocks.samples)
+    clocks.samples = []
+    # clocks: the timed region is usually shorter than NVML's update period, so
+    # the same graph is replayed for about 0.3 s right after it while the
+    # sampler runs; both sets of samples are reported
+    window = []
+    if clocks.ok:
+        clocks.start()
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < 0.3:
+            timed.replay()
+            torch.cuda.synchronize()
+        clocks.pause()
+        window = list(clocks.samples)
+        clocks.samples = []
+    del timed
+
+    # per-kernel launch times, back to back over the replicas (the same
+    # conditions as inside the step), and for comparison a launch isolated by
+    # an L2 flush and its own events
+    flush_buf = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush():
+        flush_buf.sum()
+
+    nk = max(K, 64)
+    t_fwd = backtoback_time(lambda r: (lambda: api.birkhoff_fwd(As[r], "newton", out=Ps[r])), REPLICAS, nk, stream)
+    t_bwd = backtoback_time(lambda r: (lambda: api.birkhoff_bwd(Gs[r], P=Ps[r], out=dls[r])), REPLICAS, nk, stream)
+    t_fwd_iso = event_time(lambda: api.birkhoff_fwd(A, "newton", out=P), 50, stream, flush)
+    t_bwd_iso = event_time(lambda: api.birkhoff_bwd(G, P=P, out=dl), 50, stream, flush)
+    t_step_iso = event_time(lambda: (api.birkhoff_fwd(A, "newton", out=P), api.birkhoff_bwd(G, P=P, out=dl)),
+                            50, stream, flush)
 
     _, its = api.birkhoff_fwd_diag(A)
     itf = its.float()
     newton_iters = {"mean": float(itf.mean()), "max": int(its.max()),
                     "warp_max_mean": float(itf.reshape(-1, 32).max(1).values.mean())}
+    api.birkhoff_fwd(A, "newton", out=P)
+    polished = near_permutation_fraction(P)
 
-    # end to end through the public API, host buffers, copies timed
+    # end to end through the C ABI with pinned host buffers: the native
+    # pipeline uploads, projects, differentiates and downloads in pieces
     A_h = A.cpu().pin_memory()
     G_h = G.cpu().pin_memory()
     P_h = torch.empty_like(A_h).pin_memory()
     dl_h = torch.empty_like(A_h).pin_memory()
-    A_d = torch.empty_like(A)
-    G_d = torch.empty_like(G)
-    e2e_steps = max(3, min(K, 200))
+    work = [torch.empty_like(A) for _ in range(4)]
+    pieces = args.e2e_pieces
+
+    def e2e_step():
+        api.birkhoff_fwd_bwd_host(A_h, G_h, P_h, dl_h, work, pieces)
+
+    e2e_steps = max(3, min(K, 50))
     for _ in range(3):
-        A_d.copy_(A_h, non_blocking=True)
+        e2e_step()
     torch.cuda.synchronize()
-    # the batch goes through in E2E_CHUNKS pieces on three streams, so that the
-    # upload of a piece, the kernels of the previous one and the download of the
-    # one before overlap (PCIe carries both directions at once)
-    s_in = torch.cuda.Stream(dev)
-    s_out = torch.cuda.Stream(dev)
-    bounds = [N_MATS * c // E2E_CHUNKS for c in range(E2E_CHUNKS + 1)]
-
-    def pipelined_step(start):
-        s_in.wait_event(start)
-        for c in range(E2E_CHUNKS):
-            lo, hi = bounds[c], bounds[c + 1]
-            with torch.cuda.stream(s_in):
-                A_d[lo:hi].copy_(A_h[lo:hi], non_blocking=True)
-                G_d[lo:hi].copy_(G_h[lo:hi], non_blocking=True)
-                landed = torch.cuda.Event()
-                landed.record(s_in)
-            stream.wait_event(landed)
-            api.birkhoff_fwd(A_d[lo:hi], "newton", out=P[lo:hi])
-            api.birkhoff_bwd(G_d[lo:hi], P=P[lo:hi], out=dl[lo:hi])
-            computed = torch.cuda.Event()
-            computed.record(stream)
-            s_out.wait_event(computed)
-            with torch.cuda.stream(s_out):
-                P_h[lo:hi].copy_(P[lo:hi], non_blocking=True)
-                dl_h[lo:hi].copy_(dl[lo:hi], non_blocking=True)
-        fin = torch.cuda.Event()
-        fin.record(s_out)
-        stream.wait_event(fin)
-
     tot = 0.0
     for i in range(e2e_steps):
-        flush()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        pipelined_step(e0)
-        e1.record(stream)
-        e1.synchronize()
-        tot += e0.elapsed_time(e1) * 1e-3
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        e2e_step()
+        f1.record(stream)
+        f1.synchronize()
+        tot += f0.elapsed_time(f1) * 1e-3
     t_e2e = max_over_ranks(tot / e2e_steps, pg, dev)
-    # one more step with the device inputs poisoned first: a kernel that read its
-    # inputs before their upload landed would leave NaN in the host results
-    A_d.fill_(float("nan"))
-    G_d.fill_(float("nan"))
+    # one more step with the device staging poisoned first: a kernel that read
+    # its inputs before their upload landed would leave NaN in the host results
+    for w in work:
+        w.fill_(float("nan"))
     P_h.zero_()
     dl_h.zero_()
-    start = torch.cuda.Event()
-    start.record(stream)
-    pipelined_step(start)
+    e2e_step()
     torch.cuda.synchronize()
     api.birkhoff_fwd(A, "newton", out=P)
     api.birkhoff_bwd(G, P=P, out=dl)
     matches = bool(torch.equal(dl_h, dl.cpu()) and torch.equal(P_h, P.cpu()))
-    e2e = {"value": world * N_MATS / t_e2e, "unit": UNIT, "h2d_bytes_per_step": 2 * A.numel() * 4,
-           "d2h_bytes_per_step": 2 * A.numel() * 4,
-           "path": "pinned host -> device copies, Newton fwd, implicit bwd, device -> host copies of P and "
-                   "dlogits, in %d pieces overlapped on three streams" % E2E_CHUNKS,
+    nbytes = 2 * A.numel() * 4
+    e2e = {"value": world * N_MATS / t_e2e, "unit": UNIT, "h2d_bytes_per_step": nbytes,
+           "d2h_bytes_per_step": nbytes, "ms_per_step": t_e2e * 1e3,
+           "h2d_gbs": nbytes / t_e2e / 1e9, "d2h_gbs": nbytes / t_e2e / 1e9,
+           "path": "mhc_birkhoff_fwd_bwd_host (C ABI): pinned host -> device copies, Newton fwd, implicit bwd, "
+                   "device -> host copies of P and dlogits, in %d pieces on two copy streams and the "
+                   "launching stream" % pieces,
            "matches_device_run": matches}
 
-    # dominant kernel and its roofline (HBM-bound: algorithmic bytes / time)
+    # dominant kernel and its roofline
+    mhz = clocks.max_mhz or 1965
     if t_fwd >= t_bwd:
-        kname, kbytes, kt = "newton_fwd_kernel", BYTES_FWD * N_MATS, t_fwd / K
+        kname, kt = "newton_fwd_kernel", t_fwd
+        bound, roofs = projection_roofline("newton_fwd", N_MATS, kt, hbm, mhz, newton_iters["mean"], polished)
+        kt_iso = t_fwd_iso
     else:
-        kname, kbytes, kt = "implicit_bwd_kernel", BYTES_BWD * N_MATS, t_bwd / K
-    achieved = kbytes / kt / 1e9
+        kname, kt = "implicit_bwd_kernel", t_bwd
+        bound, roofs = projection_roofline("implicit_bwd", N_MATS, kt, hbm, mhz)
+        kt_iso = t_bwd_iso
+    top = roofs[bound]
     traffic = profiled_traffic(kname)
-    roofline = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                "frac": achieved / hbm, "traffic": traffic, "peak_source": hbm_src,
-                "algorithmic_bytes_per_launch": kbytes, "launch_us": kt * 1e6,
-                "note": "peak is the %s HBM copy bandwidth; the kernel is timed in isolation" % hbm_src}
-    if kname == "newton_fwd_kernel":
-        roofline["note"] += (". %d matrices are one wave of threads, so the launch lasts as long as its slowest "
-                             "warps (Newton iterations: max %d, per-warp maximum %.2f on average, mean %.2f): "
-                             "latency- and tail-bound, not bandwidth-bound; the large-batch fractions of the "
-                             "same kernel are in extras.sweep"
-                             % (N_MATS, newton_iters["max"], newton_iters["warp_max_mean"], newton_iters["mean"]))
+    roofline = {"bound": "hbm" if bound == "hbm" else "alu", "achieved": top["achieved"], "peak": top["peak"],
+                "unit": top["unit"], "frac": top["frac"], "traffic": traffic, "kernel": kname,
+                "peak_source": {"hbm": hbm_src, "fp32": "148 SMs x 128 lanes x %d MHz" % mhz,
+                                "mufu": "148 SMs x 16 lanes x %d MHz" % mhz}[bound],
+                "launch_us": kt * 1e6, "launch_us_isolated": kt_iso * 1e6,
+                "roofs": {k: {"frac": v["frac"], "min_us": v["min_us"], "achieved": v["achieved"],
+                              "peak": v["peak"], "unit": v["unit"], "work_per_launch": v["work_per_launch"]}
+                          for k, v in roofs.items()},
+                "note": "launch_us is the mean of back-to-back launches over the rotating replicas (a CUDA graph, "
+                        "the conditions inside the step); launch_us_isolated is one launch between an L2 flush "
+                        "and its own events, which adds the launch latency. hbm peak: the %s copy bandwidth; "
+                        "fp32/mufu: the method's executed work at the measured mean of %.2f Newton iterations "
+                        "(per-warp maximum %.2f, %.1f%% of matrices taking the near-permutation step)"
+                        % (hbm_src, newton_iters["mean"], newton_iters["warp_max_mean"], 100 * polished)}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": 1e3 * t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "n_mats_per_gpu": N_MATS,
-                   "logits": "first half N(0,1), second half N(0,10^2), seed 2 (+7919*rank)",
-                   "step": "Newton fwd (to max|colsum-1|<1e-6) + implicit bwd",
-                   "l2": "flushed (512 MiB read) before every step, outside its events",
-                   "parallelism": "token-sharded replicas, no collective" if world > 1 else "single GPU"},
-        "fwd_matrices_per_s": world * N_MATS * K / max_over_ranks(t_fwd, pg, dev),
-        "bwd_matrices_per_s": world * N_MATS * K / max_over_ranks(t_bwd, pg, dev),
-        "newton_iters": newton_iters,
+        "dtype": "f32", "data": "synthetic", "config": headline_config(world),
+        "fwd_matrices_per_s": world * N_MATS / max_over_ranks(t_fwd, pg, dev),
+        "bwd_matrices_per_s": world * N_MATS / max_over_ranks(t_bwd, pg, dev),
+        "step_us_isolated": t_step_iso * 1e6,
+        "newton_iters": newton_iters, "near_permutation_step_fraction": polished,
         "e2e": e2e, "gpu_launches": gpu_launches, "roofline": roofline,
     }
-
-    line["clocks"] = clocks.summary()
+    cl = clocks.summary(window + in_region)
+    cl["samples_in_timed_region"] = len(in_region)
+    cl["window"] = ("NVML every 2 ms during the timed region (%.2f ms) and over a 0.3 s replay of the same K-step "
+                    "graph right after it" % (t_step * 1e3))
+    line["config"]["graph_uploaded_before_timing"] = uploaded
+    line["clocks"] = cl
     # the extras characterise one GPU; under torchrun the other ranks would sit in
     # the closing barrier meanwhile, so they run only when there is one rank
     if world == 1 and not args.no_extras:
         clocks.samples = []
         clocks.start()
         try:
-            line["extras"] = extras(dev, stream, flush, hbm, api, inputs)
-            # SK-20 on the default workload, for comparison
+            line["extras"] = extras(dev, stream, flush, hbm, mhz, api, inputs)
             tsk = event_time(lambda: api.birkhoff_fwd(A, "sinkhorn", 20, out=P), 20, stream, flush)
             line["extras"]["sinkhorn20_default_workload_matrices_per_s"] = N_MATS / tsk
         finally:
@@ -663,6 +857,7 @@ def run_b200(args):
         line["cpu_baseline"] = cpu_oracle_rate(args.cpu_seconds)
     elif rank == 0:
         line["cpu_baseline"] = None
+    line["targets"] = targets_summary(line, hbm)
 
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -698,15 +893,19 @@ def run_profile_case(args):
         desc = {"n_mats": cnt, "n": args.n}
     elif k in ("newton_fwd", "sinkhorn_fwd", "sinkhorn_bwd", "implicit_bwd"):
         n = args.size
-        A = torch.from_numpy(inputs.birkhoff_logits(n, args.dist, 5)).to(dev)
-        G = torch.from_numpy(inputs.upstream_grad(n, 6)).to(dev)
+        if args.dist == "halves_1_10" and n == N_MATS:
+            A_np, G_np = inputs.birkhoff_workload(WORKLOAD)
+        else:
+            A_np, G_np = inputs.birkhoff_logits(n, args.dist, 5), inputs.upstream_grad(n, 6)
+        A = torch.from_numpy(A_np).to(dev)
+        G = torch.from_numpy(G_np).to(dev)
         P = api.birkhoff_fwd(A, "newton")
         out = torch.empty_like(A)
-        fn = {"newton_fwd": lambda: api.birkhoff_fwd(A, "newton", out=out),
+        fn = {"newton_fwd": lambda: api.birkhoff_fwd(A, args.method, out=out),
               "sinkhorn_fwd": lambda: api.birkhoff_fwd(A, "sinkhorn", 20, out=out),
               "sinkhorn_bwd": lambda: api.sinkhorn_bwd(G, A, 20),
               "implicit_bwd": lambda: api.birkhoff_bwd(G, P=P, out=out)}[k]
-        desc = {"n_mats": n, "dist": args.dist}
+        desc = {"n_mats": n, "dist": args.dist, "method": args.method}
     else:
         m = inputs.mix_workload("mix_T16384_C4096", device=dev, T=args.size, C=args.channels)
         X, F, dY = m["X"], m["F"], m["dY"]

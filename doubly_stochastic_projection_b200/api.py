@@ -21,7 +21,9 @@ from . import build as _build
 SINKHORN = 0
 NEWTON = 1
 NEWTON_REFINED = 2
-_METHODS = {"sinkhorn": SINKHORN, "newton": NEWTON, "newton_refined": NEWTON_REFINED}
+NEWTON_ABSOLUTE = 3
+_METHODS = {"sinkhorn": SINKHORN, "newton": NEWTON, "newton_refined": NEWTON_REFINED,
+            "newton_absolute": NEWTON_ABSOLUTE}
 
 _lock = threading.Lock()
 _lib = None
@@ -68,6 +70,7 @@ def lib() -> ctypes.CDLL:
                 "mhc_residual_mix_bwd": [p, p, p, p, p, p, p, p, p, p, i64, i64, p],
                 "mhc_proj_mix_fwd": [p, p, p, p, p, p, i64, i64, i32, p],
                 "mhc_proj_mix_bwd": [p, p, p, p, p, p, p, p, p, i64, i64, p],
+                "mhc_birkhoff_fwd_bwd_host": [p, p, p, p, p, p, p, p, i64, i32, p],
             }
             for name, args in sig.items():
                 f = getattr(L, name)
@@ -122,9 +125,11 @@ def birkhoff_fwd(logits: torch.Tensor, method="newton", iters: int = 0, out: tor
     """Project [..., 4, 4] float32 logits onto the Birkhoff polytope.
 
     ``method``: "newton" (exact projection by Newton on the 3-variable reduced
-    dual; ``iters`` = maximum iterations, 0 -> 50), "newton_refined" (the same
-    plus a relative-accuracy step for matrices close to a permutation), or
-    "sinkhorn" (exactly ``iters`` Sinkhorn-Knopp rounds, 0 -> 20).
+    dual, with small entries of near-permutation matrices accurate relative to
+    themselves; ``iters`` = maximum iterations, 0 -> 100), "newton_refined"
+    (the same), "newton_absolute" (without that relative-accuracy step:
+    absolute accuracy only, for forward-only use), or "sinkhorn" (exactly
+    ``iters`` Sinkhorn-Knopp rounds, 0 -> 20).
     """
     _need(logits, "logits", torch.float32)
     n = _n_mats(logits)
@@ -161,6 +166,31 @@ def birkhoff_bwd(dP: torch.Tensor, P: torch.Tensor | None = None, logits: torch.
     _need(out, "out", torch.float32, dP.shape)
     _check(lib().mhc_birkhoff_bwd(_ptr(logits), _ptr(P), _ptr(dP), _ptr(out), n, _stream(dP)))
     return out
+
+
+def birkhoff_fwd_bwd_host(logits_h, dP_h, P_h, dlogits_h, work, pieces: int = 8):
+    """Newton forward + implicit backward of a batch in pinned host memory, the
+    copies pipelined with the kernels (mhc_birkhoff_fwd_bwd_host).
+
+    ``logits_h``, ``dP_h`` (read) and ``P_h``, ``dlogits_h`` (written) are pinned
+    CPU float32 tensors of the same [..., 4, 4] shape; ``work`` is a tuple of four
+    device tensors of that shape (staging for logits, dP, P and dlogits).  The
+    call is asynchronous on the current stream of the work tensors' device;
+    synchronise it before reading the host outputs."""
+    for name, t in (("logits_h", logits_h), ("dP_h", dP_h), ("P_h", P_h), ("dlogits_h", dlogits_h)):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous float32 CPU tensor" % name)
+        if not t.is_pinned():
+            raise ValueError("%s must be in pinned (page-locked) host memory" % name)
+        if t.shape != logits_h.shape:
+            raise ValueError("%s must have shape %s" % (name, tuple(logits_h.shape)))
+    if len(work) != 4:
+        raise ValueError("work must hold four device tensors (logits, dP, P, dlogits)")
+    for i, t in enumerate(work):
+        _need(t, "work[%d]" % i, torch.float32, logits_h.shape)
+    n = _n_mats(logits_h)
+    _check(lib().mhc_birkhoff_fwd_bwd_host(_ptr(logits_h), _ptr(dP_h), _ptr(P_h), _ptr(dlogits_h),
+                                           *[_ptr(t) for t in work], n, int(pieces), _stream(work[0])))
 
 
 def _square(t, name):

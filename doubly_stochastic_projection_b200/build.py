@@ -2,8 +2,13 @@
 
 The library is built into the package directory (next to this file) so that it
 travels with the source tree; nothing is installed elsewhere.  Flags: sm_100a
-only, -O3, line info for profilers, IEEE division/square root and no
-flush-to-zero (no fast-math), static CUDA runtime.
+only, -O3, line info for profilers, static CUDA runtime, and no --use_fast_math:
+plain C division and square root stay IEEE-rounded and ordinary fp32 arithmetic
+keeps subnormals.  The projection kernels choose approximate instructions
+explicitly where an approximation cannot move their result (the hardware
+reciprocal and base-2 exponential, which flush subnormal results to zero,
+and __expf / __logf inside the Newton step control); each such use is
+commented where it occurs.
 """
 from __future__ import annotations
 

@@ -36,8 +36,6 @@ constexpr int kMaxHalvings = 24;
 constexpr float kStepCap = 4.0f;
 // Levenberg-Marquardt damping factor (see newton_project).
 constexpr float kDamping = 0.03f;
-// Largest step (log units) the near-permutation polish may take.
-constexpr float kPolishMaxStep = 0.5f;
 
 // Reciprocal to within 1 ulp (MUFU), flushing subnormals.  Used where a
 // reciprocal only rescales an iterate (normalisations, elimination pivots):
@@ -232,51 +230,56 @@ __device__ __forceinline__ void sinkhorn_project(float (&a)[16], int iters)
 // rounding of that entry (~6e-8), so Newton stops with the small entries of
 // such a matrix accurate only in absolute terms: entries of 1e-4 are then off
 // by up to 1e-3 of their value, and so is the gradient, which scales with
-// them.  When every row has an entry >= 0.9 (at convergence these sit in
-// distinct columns, as each column sums to one), the deviation can instead be
-// formed from small numbers only, taking each row's dominant entry as one
-// minus the rest of its row:
-//     colsum_j - 1 = sum_{i: k_i != j} P_ij - sum_{k != j} P_{i*,k},
+// them.  When every row has an entry above 0.6 -- at convergence these sit in
+// distinct columns, since two of them would put a column sum above 1.2 -- the
+// deviation can instead be formed from small numbers only, taking each row's
+// dominant entry as one minus the rest of its row:
+//     colsum_j - 1 = sum_{i: P_ij < 1/2} P_ij - o_{i*},   o_i = sum_{k: P_ik < 1/2} P_ik,
 // where i* is the row whose dominant entry is in column j.  One Newton step on
 // this gradient (quadratic convergence from ~1e-3 relative error) leaves the
-// small entries accurate to about 1e-7 of their value.
+// small entries accurate to about 1e-7 of their value.  The step is skipped
+// unless some row's off-dominant mass is below 0.02 (row maximum above 0.98):
+// with more mass than that, absolute accuracy is already relative accuracy
+// to about 1e-5.  The step is capped like a Newton step (kStepCap) and kept
+// only if the result is doubly stochastic to the Newton tolerance.
 // ---------------------------------------------------------------------------
+constexpr float kPolishDominant = 0.6f;
+constexpr float kPolishNeeded = 0.98f;
+
 __device__ __forceinline__ void polish_near_permutation(float (&a)[16])
 {
     float m[4];
-    int k[4];
-    unsigned cols = 0;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const float* q = a + 4 * r;
-        m[r] = fmaxf(fmaxf(q[0], q[1]), fmaxf(q[2], q[3]));
-        k[r] = q[0] == m[r] ? 0 : q[1] == m[r] ? 1 : q[2] == m[r] ? 2 : 3;
-        cols |= 1u << k[r];
-    }
-    if (fminf(fminf(m[0], m[1]), fminf(m[2], m[3])) < 0.9f || cols != 15u) return;
+    for (int r = 0; r < 4; ++r) m[r] = fmaxf(fmaxf(a[4 * r], a[4 * r + 1]), fmaxf(a[4 * r + 2], a[4 * r + 3]));
+    const float lo = fminf(fminf(m[0], m[1]), fminf(m[2], m[3]));
+    const float hi = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+    if (!(lo > kPolishDominant && hi > kPolishNeeded)) return;
     // off-dominant mass of each row, summed without its dominant entry
     float o[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         const float* q = a + 4 * r;
-        o[r] = ((k[r] == 0 ? 0.0f : q[0]) + (k[r] == 1 ? 0.0f : q[1])) +
-               ((k[r] == 2 ? 0.0f : q[2]) + (k[r] == 3 ? 0.0f : q[3]));
+        o[r] = ((q[0] < 0.5f ? q[0] : 0.0f) + (q[1] < 0.5f ? q[1] : 0.0f)) +
+               ((q[2] < 0.5f ? q[2] : 0.0f) + (q[3] < 0.5f ? q[3] : 0.0f));
     }
     float g[3];
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
         float sum = 0.0f;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) sum += k[r] == j ? -o[r] : a[4 * r + j];
+        for (int r = 0; r < 4; ++r) sum += a[4 * r + j] < 0.5f ? a[4 * r + j] : -o[r];
         g[j] = sum;
     }
     const PairWeights w = pair_weights(a);
     float d0, d1, d2;
     if (!laplacian_solve(w, -g[0], -g[1], -g[2], d0, d1, d2)) return;
-    // A converged iterate needs only a small correction.  A long step means
-    // the Laplacian weights (products of entries) have lost their accuracy
-    // to underflow -- entries far below 1e-19 -- and the step is not used.
-    if (!(fmaxf(fmaxf(fabsf(d0), fabsf(d1)), fabsf(d2)) <= kPolishMaxStep)) return;
+    const float dmax = fmaxf(fmaxf(fabsf(d0), fabsf(d1)), fabsf(d2));
+    if (dmax > kStepCap) {
+        const float sc = kStepCap * rcp_approx(dmax);
+        d0 *= sc;
+        d1 *= sc;
+        d2 *= sc;
+    }
     const float e0 = __expf(d0), e1 = __expf(d1), e2 = __expf(d2);
     float b[16];
 #pragma unroll
@@ -288,8 +291,6 @@ __device__ __forceinline__ void polish_near_permutation(float (&a)[16])
         b[4 * r + 2] = a[4 * r + 2] * (e2 * q);
         b[4 * r + 3] = a[4 * r + 3] * q;
     }
-    // keep the polished matrix only if it is still doubly stochastic to the
-    // Newton tolerance
     float err = 0.0f;
 #pragma unroll
     for (int c = 0; c < 4; ++c)
@@ -412,13 +413,14 @@ __device__ __forceinline__ void sinkhorn_vjp(const float (&A)[16], const float (
 // proportional to the error, the step capped at kStepCap per potential, and
 // Armijo backtracking on phi while the error is large; a Sinkhorn round
 // replaces the step when the Laplacian is singular or no decrease is found.
-// With kRefine, matrices close to a permutation get one more step after
-// convergence, with a cancellation-free gradient (polish_near_permutation):
-// their small entries become accurate relative to themselves, at the cost of
-// that step (about a third of the time on near-identity inputs).
+// With kRefine (the default), matrices close to a permutation get one more
+// step after convergence, with a cancellation-free gradient
+// (polish_near_permutation): their small entries, and every gradient taken
+// through them, become accurate relative to themselves.  Without it the
+// entries are accurate to about 1e-6 in absolute terms only.
 // Returns the number of Newton iterations taken (the polish step not counted).
 // ---------------------------------------------------------------------------
-template <bool kRefine = false>
+template <bool kRefine = true>
 __device__ __forceinline__ int newton_project(float (&a)[16], int maxit)
 {
     shift_rows_by_max(a);

@@ -16,6 +16,9 @@ constexpr int64_t kMaxElems = int64_t(1) << 40;      // bf16 elements per tensor
 
 bool misaligned(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
 
+// Element-wise float access only needs the element's own alignment.
+bool misaligned4(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u) != 0; }
+
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? MHC_OK : MHC_ERR_CUDA; }
 
 int check_matrices(int64_t n_mats)
@@ -36,7 +39,7 @@ int resolve_iters(int method, int iters, int* out)
     if (iters < 0 || iters > MHC_MAX_ITERS) return MHC_ERR_ARG;
     if (method == MHC_SINKHORN)
         *out = iters == 0 ? mhc::kDefaultSinkhornIters : iters;
-    else if (method == MHC_NEWTON || method == MHC_NEWTON_REFINED)
+    else if (method == MHC_NEWTON || method == MHC_NEWTON_REFINED || method == MHC_NEWTON_ABSOLUTE)
         *out = iters == 0 ? mhc::kDefaultNewtonIters : iters;
     else
         return MHC_ERR_ARG;
@@ -74,7 +77,7 @@ int mhc_birkhoff_fwd(const float* logits, float* P, int64_t n_mats, int method, 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (method == MHC_SINKHORN) return cuda_status(mhc::launch_sinkhorn_fwd(logits, P, n_mats, it, s));
     return cuda_status(
-        mhc::launch_newton_fwd(logits, P, nullptr, n_mats, it, method == MHC_NEWTON_REFINED, s));
+        mhc::launch_newton_fwd(logits, P, nullptr, n_mats, it, method != MHC_NEWTON_ABSOLUTE, s));
 }
 
 int mhc_birkhoff_fwd_diag(const float* logits, float* P, int32_t* iters_out, int64_t n_mats, int iters,
@@ -88,7 +91,7 @@ int mhc_birkhoff_fwd_diag(const float* logits, float* P, int32_t* iters_out, int
     if (!logits || !P || !iters_out) return MHC_ERR_NULL;
     if (misaligned(logits) || misaligned(P) || misaligned(iters_out)) return MHC_ERR_ALIGN;
     return cuda_status(
-        mhc::launch_newton_fwd(logits, P, iters_out, n_mats, it, false, static_cast<cudaStream_t>(stream)));
+        mhc::launch_newton_fwd(logits, P, iters_out, n_mats, it, true, static_cast<cudaStream_t>(stream)));
 }
 
 int mhc_birkhoff_bwd(const float* logits, const float* P, const float* dP, float* dlogits, int64_t n_mats,
@@ -108,15 +111,15 @@ int mhc_birkhoff_fwd_n(const float* logits, float* P, int64_t n_mats, int n, int
     if (n < 1 || n > 8) return MHC_ERR_SIZE;
     int rc = check_matrices(n_mats);
     if (rc != MHC_OK) return rc;
-    if (method == MHC_NEWTON_REFINED && n != 4) return MHC_ERR_ARG;
+    if ((method == MHC_NEWTON_REFINED || method == MHC_NEWTON_ABSOLUTE) && n != 4) return MHC_ERR_ARG;
     int it = 0;
     if ((rc = resolve_iters(method, iters, &it)) != MHC_OK) return rc;
     if (n_mats == 0) return MHC_OK;
     if (!logits || !P) return MHC_ERR_NULL;
     if (misaligned(logits) || misaligned(P)) return MHC_ERR_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (n == 4 && method == MHC_NEWTON_REFINED)
-        return cuda_status(mhc::launch_newton_fwd(logits, P, nullptr, n_mats, it, true, s));
+    if (n == 4 && method != MHC_SINKHORN)
+        return cuda_status(mhc::launch_newton_fwd(logits, P, nullptr, n_mats, it, method != MHC_NEWTON_ABSOLUTE, s));
     return cuda_status(mhc::launch_birkhoff_fwd_n(logits, P, n_mats, n, method != MHC_SINKHORN, it, s));
 }
 
@@ -148,6 +151,7 @@ int mhc_exp_shifted(const float* x, float* y, int64_t n, void* stream)
     if (n < 0 || n > (int64_t(1) << 40)) return MHC_ERR_SIZE;
     if (n == 0) return MHC_OK;
     if (!x || !y) return MHC_ERR_NULL;
+    if (misaligned4(x) || misaligned4(y)) return MHC_ERR_ALIGN;
     return cuda_status(mhc::launch_exp_shifted(x, y, n, static_cast<cudaStream_t>(stream)));
 }
 
@@ -266,7 +270,8 @@ int mhc_composite_gain(const float* P_layers, float* M, float* gain_rows, float*
     if (L < 1 || T < 0 || L > (int64_t(1) << 20) || T > (int64_t(1) << 36)) return MHC_ERR_SIZE;
     if (T == 0) return MHC_OK;
     if (!P_layers || !gain_rows || !gain_cols) return MHC_ERR_NULL;
-    if (misaligned(P_layers) || misaligned(M)) return MHC_ERR_ALIGN;
+    if (misaligned(P_layers) || misaligned(M) || misaligned(gain_rows) || misaligned(gain_cols))
+        return MHC_ERR_ALIGN;
     return cuda_status(
         mhc::launch_composite_gain(P_layers, M, gain_rows, gain_cols, L, T, static_cast<cudaStream_t>(stream)));
 }

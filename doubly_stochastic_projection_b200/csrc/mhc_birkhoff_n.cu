@@ -200,7 +200,7 @@ cudaError_t launch_birkhoff_fwd_n(const float* logits, float* P, int64_t n_mats,
     case 2: return launch_fwd_n<2>(logits, P, n_mats, newton, iters, s);
     case 3: return launch_fwd_n<3>(logits, P, n_mats, newton, iters, s);
     case 4:
-        return newton ? launch_newton_fwd(logits, P, nullptr, n_mats, iters, false, s)
+        return newton ? launch_newton_fwd(logits, P, nullptr, n_mats, iters, true, s)
                       : launch_sinkhorn_fwd(logits, P, n_mats, iters, s);
     case 5: return launch_fwd_n<5>(logits, P, n_mats, newton, iters, s);
     case 6: return launch_fwd_n<6>(logits, P, n_mats, newton, iters, s);

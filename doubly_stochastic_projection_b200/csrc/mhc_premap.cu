@@ -12,6 +12,7 @@
 //   pre-map           x_in[t,c] = sum_j s_j X[t,j,c],   s_j = sigmoid(h_pre[t,j])
 //   its backward      dX[t,j,c] (+)= s_j dx_in[t,c]
 //                     dh_pre[t,j]  = s_j (1 - s_j) sum_c dx_in[t,c] X[t,j,c]
+//   (s_j (1 - s_j) evaluated without cancellation, sigmoid_grad)
 //
 // In a layer's backward dY arrives first, the layer's own backward needs dF,
 // and only then is dx_in known.  The mix backward is therefore split:
@@ -40,12 +41,6 @@ __device__ __forceinline__ void load_sigmoids(const float* hpre, int64_t t, floa
     s[1] = sigmoidf(q.y);
     s[2] = sigmoidf(q.z);
     s[3] = sigmoidf(q.w);
-}
-
-// v[k] for a run-time k in 0..3 without a local-memory array access.
-__device__ __forceinline__ float pick4(const float (&v)[4], int k)
-{
-    return k == 0 ? v[0] : k == 1 ? v[1] : k == 2 ? v[2] : v[3];
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -106,10 +101,8 @@ premap_bwd_kernel(const uint4* X, const float* hpre, const uint4* dx_in, uint4* 
             }
         }
         block_sum<4>(acc, red, tot);
-        if (threadIdx.x < 4) {
-            const float sj = pick4(s, threadIdx.x);
-            dhpre[4 * t + threadIdx.x] = sj * (1.0f - sj) * tot[threadIdx.x];
-        }
+        if (threadIdx.x < 4)
+            dhpre[4 * t + threadIdx.x] = sigmoid_grad(hpre[4 * t + threadIdx.x]) * tot[threadIdx.x];
     }
 }
 
@@ -214,8 +207,7 @@ mix_premap_bwd_kernel(const uint4* X, const float* H, const float* hpre, const u
             if (dH) dH[16 * t + threadIdx.x] = tot[threadIdx.x];
         } else if (threadIdx.x < 20) {
             const int j = threadIdx.x - 16;
-            const float sj = pick4(s, j);
-            dhpre[4 * t + j] = sj * (1.0f - sj) * tot[threadIdx.x];
+            dhpre[4 * t + j] = sigmoid_grad(hpre[4 * t + j]) * tot[threadIdx.x];
         }
         if (dlogits != nullptr && threadIdx.x == 0) {
             float gH[16], out[16];

@@ -167,4 +167,16 @@ __device__ __forceinline__ void block_sum(float (&acc)[K], float* red, float* to
 // division; four per token).
 __device__ __forceinline__ float sigmoidf(float x) { return 1.0f / (1.0f + expf(-x)); }
 
+// Derivative of the sigmoid, e / (1 + e)^2 with e = exp(-|x|).  The textbook
+// s (1 - s) cancels in fp32 once s is close to one: its relative error grows
+// as 6e-8 / (1 - s), and for x above about 17 it rounds to zero while the
+// true value is about 4e-8.  This form has no subtraction, so it keeps full
+// relative accuracy for every x (the derivative is even in x).
+__device__ __forceinline__ float sigmoid_grad(float x)
+{
+    const float e = expf(-fabsf(x));
+    const float d = 1.0f + e;
+    return e / (d * d);
+}
+
 }  // namespace mhc

@@ -16,9 +16,11 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
- *    allocates nothing, frees nothing and keeps no state between calls apart
- *    from a per-device cache of the SM count.
+ *  - All tensor pointers are DEVICE pointers owned by the caller (the one
+ *    exception, mhc_birkhoff_fwd_bwd_host, also takes pinned host buffers).
+ *    The library allocates no memory, frees nothing and keeps no state
+ *    between calls apart from a per-device cache of the SM count and the two
+ *    copy streams (with their events) of mhc_birkhoff_fwd_bwd_host.
  *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
  *    NULL means the legacy default stream) and returns as soon as the work is
  *    enqueued.
@@ -74,9 +76,12 @@ enum mhc_status {
 
 /* Forward solvers. */
 enum mhc_method {
-    MHC_SINKHORN = 0,      /* fixed-count Sinkhorn-Knopp                     */
-    MHC_NEWTON = 1,        /* Newton's method on the 3-variable reduced dual */
-    MHC_NEWTON_REFINED = 2 /* Newton, then relative-accuracy refinement      */
+    MHC_SINKHORN = 0,       /* fixed-count Sinkhorn-Knopp                          */
+    MHC_NEWTON = 1,         /* Newton's method on the 3-variable reduced dual,
+                               small entries accurate relative to themselves      */
+    MHC_NEWTON_REFINED = 2, /* the same as MHC_NEWTON (kept for compatibility)     */
+    MHC_NEWTON_ABSOLUTE = 3 /* Newton without the relative-accuracy step: entries
+                               accurate to ~1e-6 in absolute terms only           */
 };
 
 /* Largest accepted iteration count for either solver. */
@@ -104,15 +109,18 @@ enum mhc_method {
  *             `iters` is the maximum Newton iteration count; 0 selects 100.
  *             Tolerance: every column sum within 1e-6 of one (rows are exact
  *             to rounding by construction), so every entry of P is accurate
- *             to about 1e-6 in absolute terms.
- *           MHC_NEWTON_REFINED: MHC_NEWTON followed, for matrices whose rows
- *             each hold an entry >= 0.9 (close to a permutation), by one
- *             Newton step on a column-sum deviation formed from the small
- *             entries only.  Those small entries -- and gradients through
- *             them -- then carry about 1e-7 relative accuracy instead of
- *             1e-6 absolute.  Costs about one extra iteration on such
- *             matrices (a third of the time on near-identity inputs), nothing
- *             measurable otherwise.
+ *             to about 1e-6 in absolute terms.  Matrices close to a
+ *             permutation (every row holds an entry above 0.6, and some row
+ *             one above 0.98) then get one more Newton step on a column-sum
+ *             deviation formed from their small entries only, so that those
+ *             entries -- and every gradient taken through them, which scales
+ *             with them -- carry about 1e-7 relative accuracy instead of
+ *             1e-6 absolute.  That step costs about one iteration on such
+ *             matrices and nothing on the others.
+ *           MHC_NEWTON_REFINED: identical to MHC_NEWTON.
+ *           MHC_NEWTON_ABSOLUTE: MHC_NEWTON without the near-permutation
+ *             step: faster on near-permutation batches, absolute accuracy
+ *             only (for forward-only use).
  *   iters   0 .. MHC_MAX_ITERS.
  *   stream  cudaStream_t or NULL.
  */
@@ -121,8 +129,9 @@ MHC_API int mhc_birkhoff_fwd(const float *logits, float *P, int64_t n_mats, int 
 
 /*
  * mhc_birkhoff_fwd_diag -- MHC_NEWTON forward that also writes, per matrix,
- * the number of Newton iterations taken (a diagnostic for tests and for the
- * roofline's executed-work count).
+ * the number of Newton iterations taken, the near-permutation step not
+ * counted (a diagnostic for tests and for the roofline's executed-work
+ * count).
  *
  *   iters_out [n_mats] int32, device, written.  Other arguments as
  *   mhc_birkhoff_fwd with method = MHC_NEWTON.
@@ -157,8 +166,9 @@ MHC_API int mhc_birkhoff_bwd(const float *logits, const float *P, const float *d
  * backward for n x n matrices, n = 1..8: other expansion rates of the
  * residual stream (the dual then has n - 1 free variables, [BA] §2.1; n = 1
  * reduces to the scalar 1, [NA]).  Same methods, tolerances and conventions
- * as mhc_birkhoff_fwd / mhc_birkhoff_bwd; MHC_NEWTON_REFINED is accepted for
- * n = 4 only.  n = 4 runs the 4 x 4 kernels.
+ * as mhc_birkhoff_fwd / mhc_birkhoff_bwd; MHC_NEWTON_REFINED and
+ * MHC_NEWTON_ABSOLUTE are accepted for n = 4 only.  n = 4 runs the 4 x 4
+ * kernels.
  *
  *   logits, P, dP, dlogits  [n_mats][n][n] float, device, row-major.
  *   n  1..8 (MHC_ERR_SIZE otherwise).
@@ -178,7 +188,8 @@ MHC_API int mhc_birkhoff_bwd_n(const float *P, const float *dP, float *dlogits, 
  * x = -inf giving NaN.  Exposed so that its accuracy can be checked against a
  * reference exponential; not needed to use the projection.
  *
- *   x, y  [n] float, device (4-byte alignment suffices); y may equal x.
+ *   x, y  [n] float, device; 4-byte alignment suffices (MHC_ERR_ALIGN
+ *         otherwise); y may equal x.
  *   n     >= 0, at most 2^40.
  */
 MHC_API int mhc_exp_shifted(const float *x, float *y, int64_t n, void *stream);
@@ -317,10 +328,46 @@ MHC_API int mhc_mix_premap_bwd(const uint16_t *X, const float *H_res, const floa
  * iterations.
  *
  *   P_layers [L][T][4][4] float, read.  M [T][4][4] float, written, or NULL.
- *   gain_rows, gain_cols [T] float, written.  L >= 1.
+ *   gain_rows, gain_cols [T] float, written.  L >= 1.  Every pointer,
+ *   including gain_rows and gain_cols, must be 16-byte aligned.
  */
 MHC_API int mhc_composite_gain(const float *P_layers, float *M, float *gain_rows, float *gain_cols, int64_t L,
                                int64_t T, void *stream);
+
+/* Largest number of pieces mhc_birkhoff_fwd_bwd_host accepts. */
+#define MHC_MAX_PIECES 64
+
+/*
+ * mhc_birkhoff_fwd_bwd_host -- the projection's forward and implicit backward
+ * (as mhc_birkhoff_fwd with MHC_NEWTON followed by mhc_birkhoff_bwd with the
+ * saved P) for a batch held in pinned host memory, copies included.  The
+ * batch is cut into `pieces` contiguous pieces; the upload of a piece, the
+ * two kernels of the previous piece and the download of the one before run
+ * concurrently (PCIe carries both directions at once), on two copy streams
+ * owned by the library and on `stream`.
+ *
+ *   logits_h, dP_h    [n_mats][4][4] float, PINNED host memory, read.
+ *   P_h, dlogits_h    [n_mats][4][4] float, PINNED host memory, written.
+ *   logits_d, dP_d, P_d, dlogits_d
+ *                     [n_mats][4][4] float, device, caller-owned staging: the
+ *                     uploaded inputs and the device copies of the outputs.
+ *   pieces            1 .. MHC_MAX_PIECES (MHC_ERR_ARG otherwise); more
+ *                     pieces than matrices is treated as one per matrix.
+ *   Every pointer must be 16-byte aligned.  A host pointer that is not
+ *   page-locked (cudaHostAlloc / cudaHostRegister) returns MHC_ERR_ARG: the
+ *   pipeline's overlap needs asynchronous copies.
+ *
+ * Ordering: the call starts after all work enqueued on `stream` before it,
+ * and work enqueued on `stream` afterwards sees every output written (host
+ * outputs included, so synchronising `stream` makes P_h and dlogits_h
+ * readable).  The library creates its two copy streams and their events once
+ * per device, on the first call, and keeps them until the process exits.
+ * Calls from several host threads are serialised internally while they
+ * enqueue.
+ */
+MHC_API int mhc_birkhoff_fwd_bwd_host(const float *logits_h, const float *dP_h, float *P_h, float *dlogits_h,
+                                      float *logits_d, float *dP_d, float *P_d, float *dlogits_d,
+                                      int64_t n_mats, int pieces, void *stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 MHC_API const char *mhc_status_string(int status);

@@ -56,7 +56,7 @@ def test_validation_rejects_before_any_cuda_call(L):
     L.mhc_birkhoff_bwd.argtypes = [p, p, p, p, i64, p]
     fake = 1 << 20  # never dereferenced: every call below returns before launching
     assert L.mhc_birkhoff_fwd(fake, fake, -5, 1, 0, None) == 3
-    assert L.mhc_birkhoff_fwd(fake, fake, 10, 3, 0, None) == 4
+    assert L.mhc_birkhoff_fwd(fake, fake, 10, 4, 0, None) == 4
     assert L.mhc_birkhoff_fwd(fake, fake, 10, 0, -1, None) == 4
     assert L.mhc_birkhoff_fwd(fake, fake, 10, 1, 1001, None) == 4
     assert L.mhc_birkhoff_fwd(None, fake, 10, 1, 0, None) == 1
@@ -87,13 +87,24 @@ def test_validation_of_the_remaining_entry_points(L):
     assert L.mhc_composite_gain(fake, None, fake, fake, (1 << 20) + 1, 10, None) == 3
     assert L.mhc_composite_gain(None, None, fake, fake, 2, 10, None) == 1
     assert L.mhc_composite_gain(fake + 4, None, fake, fake, 2, 10, None) == 2
+    assert L.mhc_composite_gain(fake, None, fake + 4, fake, 2, 10, None) == 2     # gain_rows
+    assert L.mhc_composite_gain(fake, None, fake, fake + 8, 2, 10, None) == 2     # gain_cols
     assert L.mhc_composite_gain(None, None, None, None, 2, 0, None) == 0       # no tokens
     L.mhc_exp_shifted.argtypes = [p, p, i64, p]
     assert L.mhc_exp_shifted(fake, fake, -1, None) == 3
     assert L.mhc_exp_shifted(None, fake, 10, None) == 1
     assert L.mhc_exp_shifted(None, None, 0, None) == 0
+    assert L.mhc_exp_shifted(fake + 1, fake, 10, None) == 2                      # odd byte offset
+    assert L.mhc_exp_shifted(fake, fake + 2, 10, None) == 2
     L.mhc_premap_bwd.argtypes = [p, p, p, p, p, i32, i64, i64, p]
     assert L.mhc_premap_bwd(fake, fake, fake, fake, fake, 2, 4, 16, None) == 4     # accumulate is 0 or 1
+    L.mhc_birkhoff_fwd_bwd_host.argtypes = [p, p, p, p, p, p, p, p, i64, i32, p]
+    assert L.mhc_birkhoff_fwd_bwd_host(*[fake] * 8, -1, 4, None) == 3
+    assert L.mhc_birkhoff_fwd_bwd_host(*[fake] * 8, 10, 0, None) == 4            # pieces >= 1
+    assert L.mhc_birkhoff_fwd_bwd_host(*[fake] * 8, 10, 65, None) == 4           # pieces <= 64
+    assert L.mhc_birkhoff_fwd_bwd_host(*[None] * 8, 0, 4, None) == 0             # nothing to do
+    assert L.mhc_birkhoff_fwd_bwd_host(None, *[fake] * 7, 10, 4, None) == 1
+    assert L.mhc_birkhoff_fwd_bwd_host(*[fake] * 7, fake + 4, 10, 4, None) == 2
     L.mhc_residual_mix_bwd.argtypes = [p, p, p, p, p, p, p, p, p, p, i64, i64, p]
     assert L.mhc_residual_mix_bwd(fake, fake, fake, fake, fake, fake, None, None, fake, None, 1 << 36, 1 << 24,
                                   None) == 3                                    # T * 4 * C above 2^40

@@ -82,47 +82,89 @@ def test_config2_fwd_bwd_131072(orc):
 
 
 # End-to-end: GPU fwd + bwd against the oracle's fwd + bwd on the same logits.
-# This includes the fp32 forward's own error.  Plain Newton's P is accurate to
-# ~1e-6 in absolute terms; on matrices close to a permutation the gradient is
-# proportional to entries of 1e-4 or less, so its relative error is bounded by
-# that absolute error (about 1e-3 of those entries), not by the backward.  The
-# refined method makes those entries accurate relative to themselves, and the
-# stricter bar applies to it.
+# This includes the fp32 forward's own error: the gradient scales with the
+# small entries of P, so the forward must make those accurate relative to
+# themselves (the near-permutation step of MHC_NEWTON) for the gradient to
+# meet the relative bar.  Bars per method: (median per matrix, p99 per matrix,
+# batch-normalised max, per-matrix max wherever the gradient is not itself
+# below 1e-4 of the upstream gradient's scale).  "newton" is the method both
+# autograd wrappers and the fused projection + mix use; "newton_absolute"
+# gives up the relative accuracy of tiny entries for speed, and its bars say
+# how much.
 E2E_BARS = {
-    # method: (median per matrix, p99 per matrix, batch-normalised, per-matrix max where not tiny)
+    "newton": (1e-4, 1e-4, 1e-4, 1e-3),
     "newton_refined": (1e-4, 1e-4, 1e-4, 1e-3),
-    "newton": (1e-4, 5e-3, 5e-4, 1e-2),
+    "newton_absolute": (1e-4, 5e-3, 5e-4, 1e-2),
 }
+E2E_DISTS = ("normal1", "normal3", "normal10", "near_identity", "near_permutation", "halves_3_deepid")
+
+
+def _e2e_check(orc, method, dl, ref, G, dist):
+    med_bar, p99_bar, batch_bar, big_bar = E2E_BARS[method]
+    rel, scale = per_matrix_rel_err(dl, ref)
+    assert np.median(rel) <= med_bar, (method, dist, np.median(rel))
+    assert np.percentile(rel, 99) <= p99_bar, (method, dist, np.percentile(rel, 99))
+    assert np.abs(dl - ref).max() <= batch_bar * np.abs(ref).max(), (method, dist)
+    big = scale >= 1e-4 * np.abs(G).reshape(-1, 16).max(1)
+    assert rel[big].max() <= big_bar, (method, dist, rel[big].max())
 
 
 @pytest.mark.parametrize("method", sorted(E2E_BARS))
 def test_end_to_end_gradient_against_oracle_projection(orc, method):
-    med_bar, p99_bar, batch_bar, big_bar = E2E_BARS[method]
-    for dist in ("normal1", "normal3", "normal10", "near_identity", "near_permutation", "halves_3_deepid"):
+    for dist in E2E_DISTS:
         A = inputs.birkhoff_logits(8192, dist, 60)
         G = inputs.upstream_grad(8192, 61)
         P_g = api.birkhoff_fwd(to_gpu(A), method)
         dl = to_np64(api.birkhoff_bwd(to_gpu(G), P=P_g))
         ref = orc.implicit_bwd(orc.newton(A.astype(np.float64), tol=1e-13, max_iter=200), G.astype(np.float64))
-        rel, scale = per_matrix_rel_err(dl, ref)
-        assert np.median(rel) <= med_bar, (dist, np.median(rel))
-        assert np.percentile(rel, 99) <= p99_bar, (dist, np.percentile(rel, 99))
-        assert np.abs(dl - ref).max() <= batch_bar * np.abs(ref).max(), (dist, np.abs(dl - ref).max() / np.abs(ref).max())
-        # per matrix, wherever the gradient is not itself at the scale of the
-        # forward's absolute error (entries of P below ~1e-6)
-        big = scale >= 1e-4 * np.abs(G).reshape(-1, 16).max(1)
-        assert rel[big].max() <= big_bar, (dist, rel[big].max())
+        _e2e_check(orc, method, dl, ref, G, dist)
+
+
+def test_end_to_end_gradient_through_autograd_and_fused_paths(orc):
+    # the gradient a trainer receives: BirkhoffProjection, and ProjectedMix
+    # whose dlogits come from the fused forward's H_res through the fused
+    # backward (checked here through the projection it saves)
+    for dist in E2E_DISTS:
+        A = inputs.birkhoff_logits(8192, dist, 63)
+        G = inputs.upstream_grad(8192, 64)
+        ref = orc.implicit_bwd(orc.newton(A.astype(np.float64), tol=1e-13, max_iter=200), G.astype(np.float64))
+        A_g = to_gpu(A).requires_grad_(True)
+        P = api.BirkhoffProjection.apply(A_g)
+        P.backward(to_gpu(G))
+        _e2e_check(orc, "newton", to_np64(A_g.grad), ref, G, dist)
+        T, C = 8192, 8
+        h = torch.zeros((T, 4), device=dev())
+        X = torch.zeros((T, 4, C), dtype=torch.bfloat16, device=dev())
+        F = torch.zeros((T, C), dtype=torch.bfloat16, device=dev())
+        _, H = api.proj_mix_fwd(to_gpu(A), h, X, F)
+        dl = to_np64(api.birkhoff_bwd(to_gpu(G), P=H))
+        _e2e_check(orc, "newton", dl, ref, G, dist)
 
 
 def test_refined_forward_parity(orc):
-    for dist in ("normal1", "normal10", "near_identity", "near_permutation"):
-        A = inputs.birkhoff_logits(20000, dist, 62)
-        P = _newton_checks(api.birkhoff_fwd(to_gpu(A), "newton_refined"), A, orc)
-        ref = orc.newton(A.astype(np.float64), tol=1e-13, max_iter=200)
-        # entries of the refined projection are accurate relative to themselves
-        if dist in ("near_identity", "near_permutation"):
-            small = ref < 0.5
-            assert (np.abs(P - ref)[small] <= 1e-5 * ref[small] + 1e-12).all()
+    for method in ("newton", "newton_refined"):
+        for dist in ("normal1", "normal10", "near_identity", "near_permutation"):
+            A = inputs.birkhoff_logits(20000, dist, 62)
+            P = _newton_checks(api.birkhoff_fwd(to_gpu(A), method), A, orc)
+            ref = orc.newton(A.astype(np.float64), tol=1e-13, max_iter=200)
+            # entries of the projection are accurate relative to themselves
+            if dist in ("near_identity", "near_permutation"):
+                small = ref < 0.5
+                assert (np.abs(P - ref)[small] <= 1e-5 * ref[small] + 1e-12).all(), (method, dist)
+
+
+def test_absolute_method_is_the_same_solve_without_the_last_step(orc):
+    # matrices far from a permutation never take the near-permutation step,
+    # so both methods return the same bits for them
+    A = inputs.birkhoff_logits(20000, "normal1", 65)
+    A_g = to_gpu(A)
+    P = api.birkhoff_fwd(A_g, "newton")
+    Pa = api.birkhoff_fwd(A_g, "newton_absolute")
+    _newton_checks(Pa, A, orc)
+    rowmax = to_np64(Pa).max(-1)
+    far = ~((rowmax.min(1) > 0.6) & (rowmax.max(1) > 0.98))
+    assert far.mean() > 0.99
+    assert torch.equal(P[torch.from_numpy(far).to(dev())], Pa[torch.from_numpy(far).to(dev())])
 
 
 @pytest.mark.parametrize("si", range(len(inputs.SWEEP_SIZES)))
@@ -217,6 +259,24 @@ def test_argument_errors():
 # ------------------------------------------------------------ Sinkhorn backward
 
 
+# The Sinkhorn backward differentiates the fp32 forward's own iterates.  Their
+# rounding (about 6e-8 relative) enters every derivative, which is a sum of
+# O(|G|) terms, so the absolute error floor of an fp32 unrolled backward is
+# about 1e-7 |G| (an fp32 emulation against the fp64 oracle measures at most
+# 1.1e-7 |G| over k = 1, 5, 20 and four logit distributions).  The per-matrix
+# relative bar GRAD_REL_TOL therefore holds wherever the derivative is at
+# least 1e-3 |G| -- there that floor is at most 1e-4 of it -- and below that
+# the absolute error must stay under 1e-6 |G|.
+def _sk_check(dl, ref, G, what):
+    rel, scale = per_matrix_rel_err(dl, ref)
+    gs = np.abs(G).reshape(len(G), -1).max(1)
+    big = scale >= 1e-3 * gs
+    assert rel[big].max() <= GRAD_REL_TOL, (what, rel[big].max(), int(np.argmax(np.where(big, rel, 0))))
+    err = np.abs(dl - ref).reshape(len(G), -1).max(1)
+    assert (err <= 1e-6 * gs)[~big].all(), (what, (err / gs)[~big].max())
+    assert np.median(rel) <= GRAD_REL_TOL, what
+
+
 @pytest.mark.parametrize("iters", [1, 5, 20])
 def test_sinkhorn_bwd_parity(orc, iters):
     for dist in ("normal1", "normal10", "near_permutation"):
@@ -225,8 +285,7 @@ def test_sinkhorn_bwd_parity(orc, iters):
         G = inputs.upstream_grad(n, 81)
         dl = to_np64(api.sinkhorn_bwd(to_gpu(G), to_gpu(A), iters))
         ref = orc.sinkhorn_bwd(A.astype(np.float64), G.astype(np.float64), iters)
-        rel, _ = per_matrix_rel_err(dl, ref)
-        assert np.median(rel) <= GRAD_REL_TOL, (dist, iters, np.median(rel))
+        _sk_check(dl, ref, G, (dist, iters))
         assert np.abs(dl - ref).max() <= GRAD_REL_TOL * np.abs(ref).max(), (dist, iters)
         # row shifts cancel in the first row normalisation
         assert np.abs(dl.sum(-1)).max() <= 1e-5 * np.abs(dl).max()
@@ -236,6 +295,5 @@ def test_sinkhorn_fwd_bwd_config2(orc):
     A, G = inputs.birkhoff_workload("birkhoff_fwd_bwd_131072")
     dl = to_np64(api.sinkhorn_bwd(to_gpu(G), to_gpu(A), 20))
     ref = orc.sinkhorn_bwd(A.astype(np.float64), G.astype(np.float64), 20)
-    rel, _ = per_matrix_rel_err(dl, ref)
-    assert np.median(rel) <= GRAD_REL_TOL
+    _sk_check(dl, ref, G, "config2")
     assert np.abs(dl - ref).max() <= GRAD_REL_TOL * np.abs(ref).max()

@@ -51,6 +51,7 @@ def test_n4_is_the_4x4_path():
     A = to_gpu(_logits(3000, 4, 3.0, 8))
     assert torch.equal(api.birkhoff_fwd_n(A, "newton"), api.birkhoff_fwd(A, "newton"))
     assert torch.equal(api.birkhoff_fwd_n(A, "newton_refined"), api.birkhoff_fwd(A, "newton_refined"))
+    assert torch.equal(api.birkhoff_fwd_n(A, "newton_absolute"), api.birkhoff_fwd(A, "newton_absolute"))
     assert torch.equal(api.birkhoff_fwd_n(A, "sinkhorn", 7), api.birkhoff_fwd(A, "sinkhorn", 7))
 
 
@@ -61,6 +62,7 @@ def test_n_argument_errors():
     assert L.mhc_birkhoff_fwd_n(p, p, 4, 9, 1, 0, None) == 3
     assert L.mhc_birkhoff_fwd_n(p, p, 4, 0, 1, 0, None) == 3
     assert L.mhc_birkhoff_fwd_n(p, p, 4, 3, 2, 0, None) == 4   # refined is 4 x 4 only
+    assert L.mhc_birkhoff_fwd_n(p, p, 4, 3, 3, 0, None) == 4   # and so is absolute
     assert L.mhc_birkhoff_bwd_n(p, p, p, 4, 9, None) == 3
     torch.cuda.synchronize()
 

@@ -27,13 +27,16 @@ def _case(T, C, seed):
     return m, h_pre, dx_in
 
 
-@pytest.mark.parametrize("T,C,n_sample", [(1, 8, None), (5, 1040, None), (33, 4096, None), (1000, 8 * 385, None),
-                                         (16384, 4096, 24)])
-def test_premap_and_split_backward(orc, T, C, n_sample):
+@pytest.mark.parametrize("T,C,full", [(1, 8, False), (5, 1040, False), (33, 4096, False), (1000, 8 * 385, False),
+                                     (16384, 4096, True)])
+def test_premap_and_split_backward(orc, T, C, full):
     m, h_pre, dx_in = _case(T, C, 40)
     X, F, dY = m["X"], m["F"], m["dY"]
     hp = to_gpu(h_pre)
-    idx = np.arange(T) if n_sample is None else sample_indices(T, n_sample, 41)
+    # at the full size: token 0, the final grid-stride round of any persistent
+    # grid of up to 16 CTAs on each of 148 SMs, and 1024 seeded random tokens
+    idx = np.arange(T) if not full else np.unique(np.concatenate(
+        [[0], np.arange(T - 16 * 148, T), sample_indices(T, 1024, 41)]))
     Xs, dxs = bf16_bits(X[idx]), bf16_bits(dx_in[idx])
 
     x_in = api.premap_fwd(X, hp)
@@ -69,6 +72,29 @@ def test_premap_and_split_backward(orc, T, C, n_sample):
     dX_acc, _ = api.premap_bwd(X, hp, dx_in, dX=full["dX"].clone(), accumulate=True)
     _rel_ok(to_np64(out["dX"]), to_np64(dX_acc), MIX_REL_TOL)
     assert torch.equal(dF, full["dF"])
+
+
+def test_saturated_read_weights_keep_relative_accuracy(orc):
+    # |h_pre| in 8..20: the sigmoid's derivative is 4e-4 .. 2e-9, far below the
+    # rounding of 1 - sigmoid in fp32.  Each entry of dh_pre must carry the
+    # derivative to full relative accuracy; the only error left is that of the
+    # fp32 sum over C, bounded by the sum of the absolute products.
+    T, C = 64, 1024
+    m, _, dx_in = _case(T, C, 44)
+    X, dY = m["X"], m["dY"]
+    rng = np.random.default_rng(45)
+    h_pre = (rng.uniform(8.0, 20.0, (T, 4)) * rng.choice([-1.0, 1.0], (T, 4))).astype(np.float32)
+    hp = to_gpu(h_pre)
+    Xs, dxs = bf16_bits(X), bf16_bits(dx_in)
+    _, ref = orc.premap_bwd(Xs, h_pre, dxs)
+    x64 = (Xs.astype(np.uint32) << 16).view(np.float32).astype(np.float64).reshape(T, 4, C)
+    g64 = (dxs.astype(np.uint32) << 16).view(np.float32).astype(np.float64).reshape(T, 1, C)
+    sg = 1.0 / (1.0 + np.exp(-np.abs(h_pre.astype(np.float64))))
+    scale = sg * (1.0 - sg) * np.abs(x64 * g64).sum(-1)
+    H = api.birkhoff_fwd(to_gpu(m["logits"]), "newton")
+    for got in (api.premap_bwd(X, hp, dx_in)[1], api.mix_premap_bwd(X, H, hp, dY, dx_in)["dh_pre"]):
+        err = np.abs(to_np64(got) - ref)
+        assert (err <= RED_REL_TOL * scale).all(), (err / scale).max()
 
 
 def test_premap_errors():
