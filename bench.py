@@ -613,9 +613,9 @@ def extras(dev, stream, flush, hbm, mhz, api, inputs):
 
 def near_permutation_fraction(P):
     """Fraction of matrices that take the near-permutation step (every row
-    maximum above 0.6 and some row maximum above 0.98), from the output."""
+    maximum above 0.6 and some row maximum above 0.995), from the output."""
     m = P.max(-1).values
-    return float(((m.min(-1).values > 0.6) & (m.max(-1).values > 0.98)).float().mean())
+    return float(((m.min(-1).values > 0.6) & (m.max(-1).values > 0.995)).float().mean())
 
 
 def targets_summary(line, hbm):

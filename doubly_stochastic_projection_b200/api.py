@@ -56,6 +56,7 @@ def lib() -> ctypes.CDLL:
             sig = {
                 "mhc_birkhoff_fwd": [p, p, i64, i32, i32, p],
                 "mhc_birkhoff_fwd_diag": [p, p, p, i64, i32, p],
+                "mhc_birkhoff_fwd_layout": [p, p, i64, i32, i32, i32, p],
                 "mhc_birkhoff_bwd": [p, p, p, p, i64, p],
                 "mhc_sinkhorn_bwd": [p, p, p, i64, i32, p],
                 "mhc_exp_shifted": [p, p, i64, p],
@@ -138,6 +139,25 @@ def birkhoff_fwd(logits: torch.Tensor, method="newton", iters: int = 0, out: tor
     _need(out, "out", torch.float32, logits.shape)
     m = _METHODS.get(method, -1) if not isinstance(method, int) else method
     _check(lib().mhc_birkhoff_fwd(_ptr(logits), _ptr(out), n, int(m), int(iters), _stream(logits)))
+    return out
+
+
+LAYOUTS = {"auto": 0, "thread": 1, "row_group": 2}
+
+
+def birkhoff_fwd_layout(logits: torch.Tensor, layout="auto", method="newton", iters: int = 0,
+                        out: torch.Tensor | None = None):
+    """birkhoff_fwd with an explicit thread layout ("auto", "thread", or
+    "row_group": four lanes per matrix), for measuring the layouts."""
+    _need(logits, "logits", torch.float32)
+    n = _n_mats(logits)
+    if out is None:
+        out = torch.empty_like(logits)
+    _need(out, "out", torch.float32, logits.shape)
+    m = _METHODS.get(method, -1) if not isinstance(method, int) else method
+    lay = LAYOUTS.get(layout, -1) if not isinstance(layout, int) else layout
+    _check(lib().mhc_birkhoff_fwd_layout(_ptr(logits), _ptr(out), n, int(m), int(iters), int(lay),
+                                         _stream(logits)))
     return out
 
 

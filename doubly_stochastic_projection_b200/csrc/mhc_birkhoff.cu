@@ -16,6 +16,8 @@
 
 #include "birkhoff_math.cuh"
 #include "launch.h"
+#include "newton_rowgroup.cuh"
+#include "newton_x2.cuh"
 #include "pdl.cuh"
 
 namespace mhc {
@@ -39,7 +41,7 @@ sinkhorn_fwd_kernel(const float* logits, float* P, int64_t n, int iters)
     for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
         float a[16];
         load16(logits + 16 * m, a);
-        sinkhorn_project(a, iters);
+        sinkhorn_project_x2(a, iters);
         store16(P + 16 * m, a);
     }
 }
@@ -54,9 +56,29 @@ newton_fwd_kernel(const float* logits, float* P, int32_t* iters_out, int64_t n, 
     for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
         float a[16];
         load16(logits + 16 * m, a);
-        const int it = newton_project<kRefine>(a, maxit);
+        const int it = newton_project_x2<kRefine>(a, maxit);
         store16(P + 16 * m, a);
         if (kDiag) iters_out[m] = it;
+    }
+}
+
+// The same projection with four lanes per matrix, one row per lane
+// (newton_rowgroup.cuh): the layout of the Birkhoff-acceleration summary's
+// kernel at a group size of 4, kept for the layout comparison.
+template <bool kRefine>
+__global__ void __launch_bounds__(kProjThreads)
+newton_fwd_rowgroup_kernel(const float* logits, float* P, int64_t n, int maxit)
+{
+    pdl_wait();
+    pdl_trigger();
+    const RowGroup g = row_group();
+    const int q = threadIdx.x & 3;
+    const int64_t stride = ((int64_t)gridDim.x * blockDim.x) >> 2;
+    for (int64_t m = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 2; m < n; m += stride) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(logits + 16 * m) + q);
+        float a[4] = {v.x, v.y, v.z, v.w};
+        newton_project_rg<kRefine>(g, a, maxit);
+        reinterpret_cast<float4*>(P + 16 * m)[q] = make_float4(a[0], a[1], a[2], a[3]);
     }
 }
 
@@ -73,7 +95,7 @@ implicit_bwd_kernel(const float* logits, const float* P, const float* dP, float*
         float p[16], g[16], out[16];
         if (kRecompute) {
             load16(logits + 16 * m, p);
-            newton_project(p, kDefaultNewtonIters);
+            newton_project_x2(p, kDefaultNewtonIters);
         } else {
             load16(P + 16 * m, p);
         }
@@ -172,6 +194,17 @@ cudaError_t launch_newton_fwd(const float* logits, float* P, int32_t* iters_out,
                       : launch_newton<true, false>(logits, P, iters_out, n, maxit, s);
     return refine ? launch_newton<false, true>(logits, P, nullptr, n, maxit, s)
                   : launch_newton<false, false>(logits, P, nullptr, n, maxit, s);
+}
+
+cudaError_t launch_newton_fwd_rowgroup(const float* logits, float* P, int64_t n, int maxit, bool refine,
+                                       cudaStream_t s)
+{
+    if (refine) {
+        const Launch L = projection_launch((const void*)newton_fwd_rowgroup_kernel<true>, 4 * n);
+        return launch_pdl(newton_fwd_rowgroup_kernel<true>, L.grid, L.threads, 0, s, logits, P, n, maxit);
+    }
+    const Launch L = projection_launch((const void*)newton_fwd_rowgroup_kernel<false>, 4 * n);
+    return launch_pdl(newton_fwd_rowgroup_kernel<false>, L.grid, L.threads, 0, s, logits, P, n, maxit);
 }
 
 cudaError_t launch_implicit_bwd(const float* logits, const float* P, const float* dP, float* dlogits,

@@ -111,7 +111,7 @@ enum mhc_method {
  *             to rounding by construction), so every entry of P is accurate
  *             to about 1e-6 in absolute terms.  Matrices close to a
  *             permutation (every row holds an entry above 0.6, and some row
- *             one above 0.98) then get one more Newton step on a column-sum
+ *             one above 0.995) then get one more Newton step on a column-sum
  *             deviation formed from their small entries only, so that those
  *             entries -- and every gradient taken through them, which scales
  *             with them -- carry about 1e-7 relative accuracy instead of
@@ -126,6 +126,30 @@ enum mhc_method {
  */
 MHC_API int mhc_birkhoff_fwd(const float *logits, float *P, int64_t n_mats, int method, int iters,
                      void *stream);
+
+/* Thread layouts of the Newton forward (mhc_birkhoff_fwd_layout). */
+enum mhc_layout {
+    MHC_LAYOUT_AUTO = 0,     /* the library's choice: the thread-per-matrix kernel  */
+    MHC_LAYOUT_THREAD = 1,   /* one thread per matrix                               */
+    MHC_LAYOUT_ROW_GROUP = 2 /* four lanes per matrix, one row each (Newton only)  */
+};
+
+/*
+ * mhc_birkhoff_fwd_layout -- mhc_birkhoff_fwd with an explicit thread layout,
+ * for measuring the layouts against each other.  Both compute the same
+ * projection (to the same tolerances; the summation order of column sums
+ * differs, so results may differ in the last bits).  The row group is the
+ * lane-group layout of the Birkhoff-acceleration summary ([BA] §2.3: a matrix
+ * on a group of lanes, column sums by __shfl_xor_sync) at four lanes per
+ * matrix; the thread-per-matrix kernel is faster at every measured size and
+ * is what mhc_birkhoff_fwd runs.
+ *
+ *   layout  MHC_LAYOUT_AUTO, MHC_LAYOUT_THREAD or MHC_LAYOUT_ROW_GROUP
+ *           (MHC_ERR_ARG otherwise, and for MHC_LAYOUT_ROW_GROUP with
+ *           MHC_SINKHORN).  Other arguments as mhc_birkhoff_fwd.
+ */
+MHC_API int mhc_birkhoff_fwd_layout(const float *logits, float *P, int64_t n_mats, int method, int iters,
+                                    int layout, void *stream);
 
 /*
  * mhc_birkhoff_fwd_diag -- MHC_NEWTON forward that also writes, per matrix,
