@@ -13,11 +13,11 @@
 // backward that follows it overlap their launch gap.
 #include <algorithm>
 #include <atomic>
+#include <mutex>
 
 #include "birkhoff_math.cuh"
 #include "launch.h"
 #include "newton_rowgroup.cuh"
-#include "newton_x2.cuh"
 #include "pdl.cuh"
 
 namespace mhc {
@@ -36,12 +36,11 @@ __global__ void __launch_bounds__(kProjThreads)
 sinkhorn_fwd_kernel(const float* logits, float* P, int64_t n, int iters)
 {
     pdl_wait();
-    pdl_trigger();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
         float a[16];
         load16(logits + 16 * m, a);
-        sinkhorn_project_x2(a, iters);
+        sinkhorn_project(a, iters);
         store16(P + 16 * m, a);
     }
 }
@@ -51,12 +50,11 @@ __global__ void __launch_bounds__(kProjThreads)
 newton_fwd_kernel(const float* logits, float* P, int32_t* iters_out, int64_t n, int maxit)
 {
     pdl_wait();
-    pdl_trigger();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
         float a[16];
         load16(logits + 16 * m, a);
-        const int it = newton_project_x2<kRefine>(a, maxit);
+        const int it = newton_project<kRefine>(a, maxit);
         store16(P + 16 * m, a);
         if (kDiag) iters_out[m] = it;
     }
@@ -70,7 +68,6 @@ __global__ void __launch_bounds__(kProjThreads)
 newton_fwd_rowgroup_kernel(const float* logits, float* P, int64_t n, int maxit)
 {
     pdl_wait();
-    pdl_trigger();
     const RowGroup g = row_group();
     const int q = threadIdx.x & 3;
     const int64_t stride = ((int64_t)gridDim.x * blockDim.x) >> 2;
@@ -89,13 +86,12 @@ __global__ void __launch_bounds__(kProjThreads)
 implicit_bwd_kernel(const float* logits, const float* P, const float* dP, float* dlogits, int64_t n)
 {
     pdl_wait();
-    pdl_trigger();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
         float p[16], g[16], out[16];
         if (kRecompute) {
             load16(logits + 16 * m, p);
-            newton_project_x2(p, kDefaultNewtonIters);
+            newton_project(p, kDefaultNewtonIters);
         } else {
             load16(P + 16 * m, p);
         }
@@ -109,7 +105,6 @@ __global__ void __launch_bounds__(kProjThreads)
 sinkhorn_bwd_kernel(const float* logits, const float* dP, float* dlogits, int64_t n, int iters)
 {
     pdl_wait();
-    pdl_trigger();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
         float a[16], g[16], out[16];
@@ -140,7 +135,6 @@ Launch projection_launch(const void* kernel, int64_t n)
 __global__ void __launch_bounds__(kProjThreads) exp_shifted_kernel(const float* x, float* y, int64_t n)
 {
     pdl_wait();
-    pdl_trigger();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) y[i] = exp_shifted(x[i]);
 }
@@ -162,13 +156,44 @@ int device_sm_count()
     return v;
 }
 
-int persistent_grid(const void* kernel, int threads, size_t smem, int64_t blocks_needed)
+// Resident CTAs per SM of (kernel, threads, dynamic shared memory) on the
+// current device, asked of the runtime once and then kept: the occupancy
+// query costs microseconds of host time, as much as the launch itself.
+static int blocks_per_sm(const void* kernel, int threads, size_t smem)
 {
+    struct Entry {
+        const void* kernel;
+        int dev, threads;
+        size_t smem;
+        int per_sm;
+    };
+    constexpr int kSlots = 256;
+    static Entry table[kSlots];
+    static int used = 0;
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i)
+            if (table[i].kernel == kernel && table[i].dev == dev && table[i].threads == threads &&
+                table[i].smem == smem)
+                return table[i].per_sm;
+    }
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess ||
-        per_sm <= 0)
-        per_sm = 1;
-    const int64_t full = (int64_t)per_sm * device_sm_count();
+        per_sm <= 0) {
+        cudaGetLastError();
+        return 1;  // not cached: a failed query is asked again next time
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (used < kSlots) table[used++] = {kernel, dev, threads, smem, per_sm};
+    return per_sm;
+}
+
+int persistent_grid(const void* kernel, int threads, size_t smem, int64_t blocks_needed)
+{
+    const int64_t full = (int64_t)blocks_per_sm(kernel, threads, smem) * device_sm_count();
     return (int)std::max<int64_t>(1, std::min<int64_t>(blocks_needed, full));
 }
 

@@ -75,7 +75,6 @@ __global__ void __launch_bounds__(kThreadsN)
 fwd_n_kernel(const float* logits, float* P, int64_t n, int iters)
 {
     pdl_wait();
-    pdl_trigger();
     if constexpr (!kTiled<N>) {
         const int64_t stride = (int64_t)gridDim.x * blockDim.x;
         for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
@@ -120,7 +119,6 @@ __global__ void __launch_bounds__(kThreadsN)
 implicit_bwd_n_kernel(const float* P, const float* dP, float* dlogits, int64_t n)
 {
     pdl_wait();
-    pdl_trigger();
     if constexpr (!kTiled<N>) {
         const int64_t stride = (int64_t)gridDim.x * blockDim.x;
         for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride)

@@ -19,7 +19,6 @@
 #include "birkhoff_math.cuh"
 #include "launch.h"
 #include "mix_common.cuh"
-#include "newton_x2.cuh"
 
 namespace mhc {
 
@@ -108,7 +107,7 @@ proj_mix_fwd_kernel(const float* logits, const float* hpost, const uint4* X, con
             const int64_t t = t0 + threadIdx.x;
             float a[16];
             load16(logits + 16 * t, a);
-            newton_project_x2(a, maxit);
+            newton_project(a, maxit);
             store16(Hout + 16 * t, a);
 #pragma unroll
             for (int k = 0; k < 16; ++k) sH[threadIdx.x][k] = a[k];

@@ -147,9 +147,16 @@ def test_refined_forward_parity(orc):
             A = inputs.birkhoff_logits(20000, dist, 62)
             P = _newton_checks(api.birkhoff_fwd(to_gpu(A), method), A, orc)
             ref = orc.newton(A.astype(np.float64), tol=1e-13, max_iter=200)
-            # entries of the projection are accurate relative to themselves
+            # matrices that take the near-permutation step (every row maximum
+            # above 0.6, some row maximum above 0.995; here with a margin of
+            # 1e-4 so that the kernel's own iterate surely qualifies) have
+            # their small entries accurate relative to themselves; nearly all
+            # of these two distributions do
             if dist in ("near_identity", "near_permutation"):
-                small = ref < 0.5
+                rowmax = ref.max(-1)
+                taken = (rowmax.min(1) > 0.6 + 1e-4) & (rowmax.max(1) > 0.995 + 1e-4)
+                assert taken.mean() > 0.99, (dist, taken.mean())
+                small = (ref < 0.5) & taken[:, None, None]
                 assert (np.abs(P - ref)[small] <= 1e-5 * ref[small] + 1e-12).all(), (method, dist)
 
 
