@@ -142,13 +142,14 @@ def birkhoff_fwd(logits: torch.Tensor, method="newton", iters: int = 0, out: tor
     return out
 
 
-LAYOUTS = {"auto": 0, "thread": 1, "row_group": 2}
+LAYOUTS = {"auto": 0, "thread": 1, "row_group": 2, "lane_pair": 3}
 
 
 def birkhoff_fwd_layout(logits: torch.Tensor, layout="auto", method="newton", iters: int = 0,
                         out: torch.Tensor | None = None):
-    """birkhoff_fwd with an explicit thread layout ("auto", "thread", or
-    "row_group": four lanes per matrix), for measuring the layouts."""
+    """birkhoff_fwd with an explicit thread layout ("auto", "thread",
+    "row_group": four lanes per matrix, or "lane_pair": two lanes per
+    matrix), for measuring the layouts."""
     _need(logits, "logits", torch.float32)
     n = _n_mats(logits)
     if out is None:

@@ -18,9 +18,10 @@ int persistent_grid(const void* kernel, int threads, size_t smem, int64_t blocks
 cudaError_t launch_sinkhorn_fwd(const float* logits, float* P, int64_t n, int iters, cudaStream_t s);
 cudaError_t launch_newton_fwd(const float* logits, float* P, int32_t* iters_out, int64_t n,
                               int maxit, bool refine, cudaStream_t s);
-// The Newton forward with four lanes per matrix (one row per lane).
-cudaError_t launch_newton_fwd_rowgroup(const float* logits, float* P, int64_t n, int maxit, bool refine,
-                                       cudaStream_t s);
+// The Newton forward with `lanes` (2 or 4) lanes per matrix, 4 / lanes rows
+// per lane.
+cudaError_t launch_newton_fwd_group(const float* logits, float* P, int64_t n, int maxit, bool refine, int lanes,
+                                    cudaStream_t s);
 cudaError_t launch_sinkhorn_bwd(const float* logits, const float* dP, float* dlogits, int64_t n, int iters,
                                 cudaStream_t s);
 cudaError_t launch_implicit_bwd(const float* logits, const float* P, const float* dP, float* dlogits,

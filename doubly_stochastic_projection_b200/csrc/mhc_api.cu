@@ -83,10 +83,12 @@ int mhc_birkhoff_fwd(const float* logits, float* P, int64_t n_mats, int method, 
 int mhc_birkhoff_fwd_layout(const float* logits, float* P, int64_t n_mats, int method, int iters, int layout,
                             void* stream)
 {
-    if (layout != MHC_LAYOUT_AUTO && layout != MHC_LAYOUT_THREAD && layout != MHC_LAYOUT_ROW_GROUP)
+    if (layout != MHC_LAYOUT_AUTO && layout != MHC_LAYOUT_THREAD && layout != MHC_LAYOUT_ROW_GROUP &&
+        layout != MHC_LAYOUT_LANE_PAIR)
         return MHC_ERR_ARG;
-    if (layout == MHC_LAYOUT_ROW_GROUP && method == MHC_SINKHORN) return MHC_ERR_ARG;
-    if (layout != MHC_LAYOUT_ROW_GROUP) return mhc_birkhoff_fwd(logits, P, n_mats, method, iters, stream);
+    const bool grouped = layout == MHC_LAYOUT_ROW_GROUP || layout == MHC_LAYOUT_LANE_PAIR;
+    if (grouped && method == MHC_SINKHORN) return MHC_ERR_ARG;
+    if (!grouped) return mhc_birkhoff_fwd(logits, P, n_mats, method, iters, stream);
     int rc = check_matrices(n_mats);
     if (rc != MHC_OK) return rc;
     int it = 0;
@@ -94,8 +96,9 @@ int mhc_birkhoff_fwd_layout(const float* logits, float* P, int64_t n_mats, int m
     if (n_mats == 0) return MHC_OK;
     if (!logits || !P) return MHC_ERR_NULL;
     if (misaligned(logits) || misaligned(P)) return MHC_ERR_ALIGN;
-    return cuda_status(mhc::launch_newton_fwd_rowgroup(logits, P, n_mats, it, method != MHC_NEWTON_ABSOLUTE,
-                                                       static_cast<cudaStream_t>(stream)));
+    return cuda_status(mhc::launch_newton_fwd_group(logits, P, n_mats, it, method != MHC_NEWTON_ABSOLUTE,
+                                                    layout == MHC_LAYOUT_ROW_GROUP ? 4 : 2,
+                                                    static_cast<cudaStream_t>(stream)));
 }
 
 int mhc_birkhoff_fwd_diag(const float* logits, float* P, int32_t* iters_out, int64_t n_mats, int iters,

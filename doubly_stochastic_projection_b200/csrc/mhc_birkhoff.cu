@@ -60,22 +60,33 @@ newton_fwd_kernel(const float* logits, float* P, int32_t* iters_out, int64_t n, 
     }
 }
 
-// The same projection with four lanes per matrix, one row per lane
-// (newton_rowgroup.cuh): the layout of the Birkhoff-acceleration summary's
-// kernel at a group size of 4, kept for the layout comparison.
-template <bool kRefine>
+// The same projection with a group of L lanes per matrix, 4 / L rows per
+// lane (newton_rowgroup.cuh): the layout of the Birkhoff-acceleration
+// summary's kernel at a group size of 2 or 4, for the layout comparison.
+template <int L, bool kRefine>
 __global__ void __launch_bounds__(kProjThreads)
-newton_fwd_rowgroup_kernel(const float* logits, float* P, int64_t n, int maxit)
+newton_fwd_group_kernel(const float* logits, float* P, int64_t n, int maxit)
 {
     pdl_wait();
-    const RowGroup g = row_group();
-    const int q = threadIdx.x & 3;
-    const int64_t stride = ((int64_t)gridDim.x * blockDim.x) >> 2;
-    for (int64_t m = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 2; m < n; m += stride) {
-        const float4 v = __ldg(reinterpret_cast<const float4*>(logits + 16 * m) + q);
-        float a[4] = {v.x, v.y, v.z, v.w};
-        newton_project_rg<kRefine>(g, a, maxit);
-        reinterpret_cast<float4*>(P + 16 * m)[q] = make_float4(a[0], a[1], a[2], a[3]);
+    constexpr int R = LaneGroup<L>::kRows;
+    const LaneGroup<L> g;
+    const int q = threadIdx.x & (L - 1);
+    const int64_t stride = ((int64_t)gridDim.x * blockDim.x) / L;
+    for (int64_t m = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / L; m < n; m += stride) {
+        const float4* src = reinterpret_cast<const float4*>(logits + 16 * m) + q * R;
+        float a[4 * R];
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            const float4 v = __ldg(src + k);
+            a[4 * k] = v.x;
+            a[4 * k + 1] = v.y;
+            a[4 * k + 2] = v.z;
+            a[4 * k + 3] = v.w;
+        }
+        newton_project_lg<L, kRefine>(g, a, maxit);
+        float4* dst = reinterpret_cast<float4*>(P + 16 * m) + q * R;
+#pragma unroll
+        for (int k = 0; k < R; ++k) dst[k] = make_float4(a[4 * k], a[4 * k + 1], a[4 * k + 2], a[4 * k + 3]);
     }
 }
 
@@ -221,15 +232,19 @@ cudaError_t launch_newton_fwd(const float* logits, float* P, int32_t* iters_out,
                   : launch_newton<false, false>(logits, P, nullptr, n, maxit, s);
 }
 
-cudaError_t launch_newton_fwd_rowgroup(const float* logits, float* P, int64_t n, int maxit, bool refine,
-                                       cudaStream_t s)
+template <int L, bool kRefine>
+static cudaError_t launch_group(const float* logits, float* P, int64_t n, int maxit, cudaStream_t s)
 {
-    if (refine) {
-        const Launch L = projection_launch((const void*)newton_fwd_rowgroup_kernel<true>, 4 * n);
-        return launch_pdl(newton_fwd_rowgroup_kernel<true>, L.grid, L.threads, 0, s, logits, P, n, maxit);
-    }
-    const Launch L = projection_launch((const void*)newton_fwd_rowgroup_kernel<false>, 4 * n);
-    return launch_pdl(newton_fwd_rowgroup_kernel<false>, L.grid, L.threads, 0, s, logits, P, n, maxit);
+    const Launch Lc = projection_launch((const void*)newton_fwd_group_kernel<L, kRefine>, L * n);
+    return launch_pdl(newton_fwd_group_kernel<L, kRefine>, Lc.grid, Lc.threads, 0, s, logits, P, n, maxit);
+}
+
+cudaError_t launch_newton_fwd_group(const float* logits, float* P, int64_t n, int maxit, bool refine, int lanes,
+                                    cudaStream_t s)
+{
+    if (lanes == 4)
+        return refine ? launch_group<4, true>(logits, P, n, maxit, s) : launch_group<4, false>(logits, P, n, maxit, s);
+    return refine ? launch_group<2, true>(logits, P, n, maxit, s) : launch_group<2, false>(logits, P, n, maxit, s);
 }
 
 cudaError_t launch_implicit_bwd(const float* logits, const float* P, const float* dP, float* dlogits,

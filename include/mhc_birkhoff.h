@@ -129,24 +129,25 @@ MHC_API int mhc_birkhoff_fwd(const float *logits, float *P, int64_t n_mats, int 
 
 /* Thread layouts of the Newton forward (mhc_birkhoff_fwd_layout). */
 enum mhc_layout {
-    MHC_LAYOUT_AUTO = 0,     /* the library's choice: the thread-per-matrix kernel  */
-    MHC_LAYOUT_THREAD = 1,   /* one thread per matrix                               */
-    MHC_LAYOUT_ROW_GROUP = 2 /* four lanes per matrix, one row each (Newton only)  */
+    MHC_LAYOUT_AUTO = 0,      /* the library's choice (see mhc_birkhoff_fwd_layout)   */
+    MHC_LAYOUT_THREAD = 1,    /* one thread per matrix                                */
+    MHC_LAYOUT_ROW_GROUP = 2, /* four lanes per matrix, one row each (Newton only)    */
+    MHC_LAYOUT_LANE_PAIR = 3  /* two lanes per matrix, two rows each (Newton only)    */
 };
 
 /*
  * mhc_birkhoff_fwd_layout -- mhc_birkhoff_fwd with an explicit thread layout,
- * for measuring the layouts against each other.  Both compute the same
+ * for measuring the layouts against each other.  All compute the same
  * projection (to the same tolerances; the summation order of column sums
- * differs, so results may differ in the last bits).  The row group is the
- * lane-group layout of the Birkhoff-acceleration summary ([BA] §2.3: a matrix
- * on a group of lanes, column sums by __shfl_xor_sync) at four lanes per
- * matrix; the thread-per-matrix kernel is faster at every measured size and
- * is what mhc_birkhoff_fwd runs.
+ * differs, so results may differ in the last bits).  The row group and the
+ * lane pair are the lane-group layout of the Birkhoff-acceleration summary
+ * ([BA] §2.3: a matrix on a group of lanes, column sums by __shfl_xor_sync)
+ * at four and two lanes per matrix.  MHC_LAYOUT_AUTO is what
+ * mhc_birkhoff_fwd runs.
  *
- *   layout  MHC_LAYOUT_AUTO, MHC_LAYOUT_THREAD or MHC_LAYOUT_ROW_GROUP
- *           (MHC_ERR_ARG otherwise, and for MHC_LAYOUT_ROW_GROUP with
- *           MHC_SINKHORN).  Other arguments as mhc_birkhoff_fwd.
+ *   layout  one of enum mhc_layout (MHC_ERR_ARG otherwise, and for the
+ *           grouped layouts with MHC_SINKHORN).  Other arguments as
+ *           mhc_birkhoff_fwd.
  */
 MHC_API int mhc_birkhoff_fwd_layout(const float *logits, float *P, int64_t n_mats, int method, int iters,
                                     int layout, void *stream);

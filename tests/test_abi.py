@@ -99,7 +99,8 @@ def test_validation_of_the_remaining_entry_points(L):
     L.mhc_premap_bwd.argtypes = [p, p, p, p, p, i32, i64, i64, p]
     assert L.mhc_premap_bwd(fake, fake, fake, fake, fake, 2, 4, 16, None) == 4     # accumulate is 0 or 1
     L.mhc_birkhoff_fwd_layout.argtypes = [p, p, i64, i32, i32, i32, p]
-    assert L.mhc_birkhoff_fwd_layout(fake, fake, 10, 1, 0, 3, None) == 4          # unknown layout
+    assert L.mhc_birkhoff_fwd_layout(fake, fake, 10, 1, 0, 4, None) == 4          # unknown layout
+    assert L.mhc_birkhoff_fwd_layout(fake, fake, 10, 0, 0, 3, None) == 4          # lane pair is Newton only
     assert L.mhc_birkhoff_fwd_layout(fake, fake, 10, 0, 0, 2, None) == 4          # row group is Newton only
     assert L.mhc_birkhoff_fwd_layout(fake, fake, -1, 1, 0, 2, None) == 3
     assert L.mhc_birkhoff_fwd_layout(None, fake, 10, 1, 0, 2, None) == 1

@@ -198,33 +198,37 @@ def test_row_group_layout_parity(orc, n):
     # same tolerances (only the summation order of the group sums differs)
     A = inputs.birkhoff_logits(n, "halves_1_10", 66 + n % 5)
     A_g = to_gpu(A)
-    for method in ("newton", "newton_absolute"):
-        P_rg = api.birkhoff_fwd_layout(A_g, "row_group", method)
-        idx = sample_indices(n, 8192, 67)
-        _newton_checks(P_rg, A, orc, idx)
-        P_t = api.birkhoff_fwd_layout(A_g, "thread", method)
-        assert (P_rg - P_t).abs().max().item() <= 4e-6
-        assert torch.equal(P_t, api.birkhoff_fwd(A_g, method))
+    for layout in ("row_group", "lane_pair"):
+        for method in ("newton", "newton_absolute"):
+            P_rg = api.birkhoff_fwd_layout(A_g, layout, method)
+            idx = sample_indices(n, 8192, 67)
+            _newton_checks(P_rg, A, orc, idx)
+            P_t = api.birkhoff_fwd_layout(A_g, "thread", method)
+            assert (P_rg - P_t).abs().max().item() <= 4e-6, layout
+            assert torch.equal(P_t, api.birkhoff_fwd(A_g, method))
     # the gradient bar holds through the row-group forward as well
     G = inputs.upstream_grad(n, 68)
-    P_rg = api.birkhoff_fwd_layout(A_g, "row_group", "newton")
-    dl = to_np64(api.birkhoff_bwd(to_gpu(G), P=P_rg))
     idx = sample_indices(n, 8192, 69)
     ref = orc.implicit_bwd(orc.newton(A[idx].astype(np.float64), tol=1e-13, max_iter=200), G[idx].astype(np.float64))
-    rel, _ = per_matrix_rel_err(dl[idx], ref)
-    assert np.percentile(rel, 99) <= GRAD_REL_TOL
+    for layout in ("row_group", "lane_pair"):
+        P_rg = api.birkhoff_fwd_layout(A_g, layout, "newton")
+        dl = to_np64(api.birkhoff_bwd(to_gpu(G), P=P_rg))
+        rel, _ = per_matrix_rel_err(dl[idx], ref)
+        assert np.percentile(rel, 99) <= GRAD_REL_TOL, layout
 
 
 def test_row_group_nonfinite_and_errors():
     A = inputs.birkhoff_logits(40, "normal1", 70)
     A[3, 1, 2] = np.nan
-    P = to_np64(api.birkhoff_fwd_layout(to_gpu(A), "row_group"))
-    bad = ~np.isfinite(P).all((1, 2))
-    assert bad[3] and bad.sum() == 1
+    for layout in ("row_group", "lane_pair"):
+        P = to_np64(api.birkhoff_fwd_layout(to_gpu(A), layout))
+        bad = ~np.isfinite(P).all((1, 2))
+        assert bad[3] and bad.sum() == 1, layout
     L = api.lib()
     X = torch.zeros((8, 4, 4), device=dev())
     assert L.mhc_birkhoff_fwd_layout(X.data_ptr(), X.data_ptr(), 8, 0, 0, 2, None) == 4   # Sinkhorn
-    assert L.mhc_birkhoff_fwd_layout(X.data_ptr(), X.data_ptr(), 8, 1, 0, 3, None) == 4   # unknown layout
+    assert L.mhc_birkhoff_fwd_layout(X.data_ptr(), X.data_ptr(), 8, 0, 0, 3, None) == 4
+    assert L.mhc_birkhoff_fwd_layout(X.data_ptr(), X.data_ptr(), 8, 1, 0, 4, None) == 4   # unknown layout
     torch.cuda.synchronize()
 
 
