@@ -81,7 +81,7 @@ def parse():
     ap.add_argument("--no-extras", action="store_true", help="skip the sweep and mix extras")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-oracle sample budget (Newton leg)")
-    ap.add_argument("--e2e-pieces", type=int, default=8, help="pieces of the end-to-end host pipeline")
+    ap.add_argument("--e2e-pieces", type=int, default=4, help="pieces of the end-to-end host pipeline")
     ap.add_argument("--profile", default=None,
                     choices=["newton_fwd", "sinkhorn_fwd", "sinkhorn_bwd", "implicit_bwd", "mix_fwd", "mix_bwd",
                              "proj_mix_fwd", "proj_mix_bwd", "premap_fwd", "mix_post_bwd", "mix_premap_bwd",
@@ -508,6 +508,22 @@ def extras(dev, stream, flush, hbm, mhz, api, inputs):
                                           "fwd_frac_hbm": BYTES_FWD * n / ts / 1e9 / hbm})
             del A, G, P, dl, its
             torch.cuda.empty_cache()
+    # Thread layouts of the Newton forward (thread per matrix, lane pair, row
+    # group), back to back over rotating replicas
+    out["layouts"] = []
+    for n, dist, seed, R, L in ((131072, "halves_1_10", 2, 16, 32), (1 << 20, "normal1", 300, 4, 8),
+                                (1 << 20, "normal10", 302, 4, 8)):
+        A = torch.from_numpy(inputs.birkhoff_logits(n, dist, seed)).to(dev)
+        As = [A.clone() for _ in range(R)]
+        Ps = [torch.empty_like(A) for _ in range(R)]
+        row = {"n_mats": n, "dist": dist}
+        for lay in ("thread", "lane_pair", "row_group"):
+            t = backtoback_time(lambda r, lay=lay: (lambda: api.birkhoff_fwd_layout(As[r], lay, "newton", out=Ps[r])),
+                                R, L, stream)
+            row[lay + "_us"] = t * 1e6
+        out["layouts"].append(row)
+        del A, As, Ps
+        torch.cuda.empty_cache()
     # The pages' comparison (Birkhoff-acceleration summary, section 4): forward +
     # backward of the Newton projection with the implicit backward, against
     # 20-round Sinkhorn with the backward through the unrolled iteration.
@@ -644,6 +660,11 @@ def targets_summary(line, hbm):
                             "fused_fwd": round(r["fused_fwd_frac_hbm"], 3),
                             "fused_bwd": round(r["fused_bwd_frac_hbm"], 3),
                             "fused_fwd_bwd_tokens_per_s": round(r["fused_fwd_bwd_tokens_per_s"])}
+    if ex.get("layouts"):
+        t["newton_fwd_layout_us"] = {"%s_%s" % (size_name.get(r["n_mats"], r["n_mats"]), short.get(r["dist"], "halves")):
+                                     [round(r["thread_us"], 1), round(r["lane_pair_us"], 1), round(r["row_group_us"], 1)]
+                                     for r in ex["layouts"]}
+        t["newton_fwd_layout_order"] = "thread, lane_pair, row_group"
     rl = line.get("roofline", {})
     t["headline"] = {"matrices_per_s": round(line["value"]), "e2e_matrices_per_s": round(line["e2e"]["value"]),
                      "dominant_kernel": rl.get("kernel"), "bound": rl.get("bound"),

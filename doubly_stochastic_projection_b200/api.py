@@ -189,7 +189,7 @@ def birkhoff_bwd(dP: torch.Tensor, P: torch.Tensor | None = None, logits: torch.
     return out
 
 
-def birkhoff_fwd_bwd_host(logits_h, dP_h, P_h, dlogits_h, work, pieces: int = 8):
+def birkhoff_fwd_bwd_host(logits_h, dP_h, P_h, dlogits_h, work, pieces: int = 4):
     """Newton forward + implicit backward of a batch in pinned host memory, the
     copies pipelined with the kernels (mhc_birkhoff_fwd_bwd_host).
 

@@ -129,7 +129,7 @@ MHC_API int mhc_birkhoff_fwd(const float *logits, float *P, int64_t n_mats, int 
 
 /* Thread layouts of the Newton forward (mhc_birkhoff_fwd_layout). */
 enum mhc_layout {
-    MHC_LAYOUT_AUTO = 0,      /* the library's choice (see mhc_birkhoff_fwd_layout)   */
+    MHC_LAYOUT_AUTO = 0,      /* the library's choice: one thread per matrix          */
     MHC_LAYOUT_THREAD = 1,    /* one thread per matrix                                */
     MHC_LAYOUT_ROW_GROUP = 2, /* four lanes per matrix, one row each (Newton only)    */
     MHC_LAYOUT_LANE_PAIR = 3  /* two lanes per matrix, two rows each (Newton only)    */
@@ -142,8 +142,9 @@ enum mhc_layout {
  * differs, so results may differ in the last bits).  The row group and the
  * lane pair are the lane-group layout of the Birkhoff-acceleration summary
  * ([BA] §2.3: a matrix on a group of lanes, column sums by __shfl_xor_sync)
- * at four and two lanes per matrix.  MHC_LAYOUT_AUTO is what
- * mhc_birkhoff_fwd runs.
+ * at four and two lanes per matrix.  One thread per matrix measured fastest
+ * on B200 at every batch size and logit distribution tried (131072 to 16M
+ * matrices), so MHC_LAYOUT_AUTO -- and mhc_birkhoff_fwd -- runs it.
  *
  *   layout  one of enum mhc_layout (MHC_ERR_ARG otherwise, and for the
  *           grouped layouts with MHC_SINKHORN).  Other arguments as
