@@ -88,6 +88,8 @@ def parse():
                              "newton_fwd_n", "implicit_bwd_n", "composite_gain"],
                     help="run one kernel --reps times on one case (for ncu) and exit")
     ap.add_argument("--method", default="newton", help="--profile newton_fwd: projection method")
+    ap.add_argument("--layout", default="auto", choices=["auto", "thread", "lane_pair", "row_group"],
+                    help="--profile newton_fwd: thread layout of the Newton forward")
     ap.add_argument("--size", type=int, default=1 << 22, help="--profile: matrices, or tokens T for the mix")
     ap.add_argument("--channels", type=int, default=4096, help="--profile: mix channels C")
     ap.add_argument("--dist", default="normal1", help="--profile: logit distribution")
@@ -474,17 +476,23 @@ def extras(dev, stream, flush, hbm, mhz, api, inputs):
     out = {"sweep": [], "sinkhorn20": [], "mix": []}
     reps = 5
     for si, n in enumerate(inputs.SWEEP_SIZES):
+        # back to back over replicas whose inputs and outputs together exceed
+        # the L2 several times (as the headline step)
+        R, L = (4, 16) if n <= (1 << 20) else (2, 8)
         for di, dist in enumerate(inputs.SWEEP_DISTS):
             A = torch.from_numpy(inputs.birkhoff_logits(n, dist, inputs.sweep_seed(si, di))).to(dev)
             G = torch.from_numpy(inputs.upstream_grad(n, inputs.sweep_seed(si, di) + 1000)).to(dev)
-            P = torch.empty_like(A)
-            dl = torch.empty_like(A)
-            api.birkhoff_fwd(A, "newton", out=P)
+            As, Gs = [A] + [A.clone() for _ in range(R - 1)], [G] + [G.clone() for _ in range(R - 1)]
+            Ps, Ds = [torch.empty_like(A) for _ in range(R)], [torch.empty_like(A) for _ in range(R)]
+            for r in range(R):
+                api.birkhoff_fwd(As[r], "newton", out=Ps[r])
+            P, dl = Ps[0], Ds[0]
             _, its = api.birkhoff_fwd_diag(A)
             pol = near_permutation_fraction(P)
-            tf = event_time(lambda: api.birkhoff_fwd(A, "newton", out=P), reps, stream, flush)
-            ta = event_time(lambda: api.birkhoff_fwd(A, "newton_absolute", out=dl), reps, stream, flush)
-            tb = event_time(lambda: api.birkhoff_bwd(G, P=P, out=dl), reps, stream, flush)
+            tf = backtoback_time(lambda r: (lambda: api.birkhoff_fwd(As[r], "newton", out=Ds[r])), R, L, stream)
+            ta = backtoback_time(lambda r: (lambda: api.birkhoff_fwd(As[r], "newton_absolute", out=Ds[r])), R, L,
+                                 stream)
+            tb = backtoback_time(lambda r: (lambda: api.birkhoff_bwd(Gs[r], P=Ps[r], out=Ds[r])), R, L, stream)
             itn = its.float()
             its_mean = float(itn.mean())
             bound, roofs = projection_roofline("newton_fwd", n, tf, hbm, mhz, its_mean, pol)
@@ -502,11 +510,12 @@ def extras(dev, stream, flush, hbm, mhz, api, inputs):
                 "newton_iters_warp_max_mean": float(itn.reshape(-1, 32).max(1).values.mean()),
             })
             if dist in ("normal1", "normal10"):
-                ts = event_time(lambda: api.birkhoff_fwd(A, "sinkhorn", 20, out=P), reps, stream, flush)
+                ts = backtoback_time(lambda r: (lambda: api.birkhoff_fwd(As[r], "sinkhorn", 20, out=Ds[r])), R, L,
+                                     stream)
                 out["sinkhorn20"].append({"n_mats": n, "dist": dist, "fwd_matrices_per_s": n / ts,
                                           "fwd_gbs": BYTES_FWD * n / ts / 1e9,
                                           "fwd_frac_hbm": BYTES_FWD * n / ts / 1e9 / hbm})
-            del A, G, P, dl, its
+            del A, G, As, Gs, Ps, Ds, P, dl, its
             torch.cuda.empty_cache()
     # Thread layouts of the Newton forward (thread per matrix, lane pair, row
     # group), back to back over rotating replicas
@@ -922,11 +931,11 @@ def run_profile_case(args):
         G = torch.from_numpy(G_np).to(dev)
         P = api.birkhoff_fwd(A, "newton")
         out = torch.empty_like(A)
-        fn = {"newton_fwd": lambda: api.birkhoff_fwd(A, args.method, out=out),
+        fn = {"newton_fwd": lambda: api.birkhoff_fwd_layout(A, args.layout, args.method, out=out),
               "sinkhorn_fwd": lambda: api.birkhoff_fwd(A, "sinkhorn", 20, out=out),
               "sinkhorn_bwd": lambda: api.sinkhorn_bwd(G, A, 20),
               "implicit_bwd": lambda: api.birkhoff_bwd(G, P=P, out=out)}[k]
-        desc = {"n_mats": n, "dist": args.dist, "method": args.method}
+        desc = {"n_mats": n, "dist": args.dist, "method": args.method, "layout": args.layout}
     else:
         m = inputs.mix_workload("mix_T16384_C4096", device=dev, T=args.size, C=args.channels)
         X, F, dY = m["X"], m["F"], m["dY"]
