@@ -69,9 +69,12 @@ __device__ __forceinline__ void tile_store(float* dst, const float* tile, int64_
 }
 
 // Forward: kNewton selects Newton (maxit = iteration limit) or Sinkhorn
-// (maxit = round count).
+// (maxit = round count).  At n = 8 the Newton forward would take 142
+// registers a thread (3 CTAs an SM); capped at 128 (4 CTAs) it measured 14%
+// faster on B200 (1714 -> 1955 GB/s at 1M N(0,1) matrices) despite a few
+// bytes of spill.  The same cap made n = 5 and the n = 8 backward slower.
 template <int N, bool kNewton>
-__global__ void __launch_bounds__(kThreadsN)
+__global__ void __launch_bounds__(kThreadsN, N == 8 ? 4 : 1)
 fwd_n_kernel(const float* logits, float* P, int64_t n, int iters)
 {
     pdl_wait();
