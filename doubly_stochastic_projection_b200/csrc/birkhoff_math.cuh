@@ -629,58 +629,4 @@ __device__ __forceinline__ void implicit_vjp(const float (&pf)[16], const float 
     }
 }
 
-// implicit_vjp for a matrix read from memory row by row (twice: once for the
-// column sums of S and the Laplacian weights, once for the result) instead of
-// held in registers, and written row by row.  The arithmetic is that of
-// implicit_vjp; only the order in which the weights are accumulated differs.
-// Holding neither P nor G whole keeps the kernel near 64 registers a thread,
-// so that a batch of 131072 matrices is one wave of resident threads.  out may
-// equal G: row r of G is read before row r of out is written and never after.
-__device__ __forceinline__ void implicit_vjp_rows(const float* P, const float* G, float* out)
-{
-    const float4* P4 = reinterpret_cast<const float4*>(P);
-    const float4* G4 = reinterpret_cast<const float4*>(G);
-    double c0 = 0.0, c1 = 0.0, c2 = 0.0;
-    PairWeightsD w = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const float4 pv = P4[r], gv = G4[r];
-        const float gr[4] = {gv.x, gv.y, gv.z, gv.w};
-        double D[6];
-        row_differences(gr, D);
-        const double q0 = pv.x, q1 = pv.y, q2 = pv.z, q3 = pv.w;
-        c0 = fma(q0, fma(q1, D[0], fma(q2, D[1], q3 * D[2])), c0);
-        c1 = fma(q1, fma(q2, D[3], fma(q3, D[4], -q0 * D[0])), c1);
-        c2 = fma(q2, fma(q3, D[5], fma(-q0, D[1], -q1 * D[3])), c2);
-        w.w01 = fma(q0, q1, w.w01);
-        w.w02 = fma(q0, q2, w.w02);
-        w.w03 = fma(q0, q3, w.w03);
-        w.w12 = fma(q1, q2, w.w12);
-        w.w13 = fma(q1, q3, w.w13);
-        w.w23 = fma(q2, q3, w.w23);
-    }
-    double l0, l1, l2;
-    const bool ok = laplacian_solve_d(w, c0, c1, c2, l0, l1, l2);
-    const double L[6] = {l0 - l1, l0 - l2, l0, l1 - l2, l1, l2};
-    float4* O4 = reinterpret_cast<float4*>(out);
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const float4 pv = P4[r], gv = G4[r];
-        const float gr[4] = {gv.x, gv.y, gv.z, gv.w};
-        double E[6];
-        row_differences(gr, E);
-#pragma unroll
-        for (int k = 0; k < 6; ++k) E[k] -= L[k];
-        const double q0 = pv.x, q1 = pv.y, q2 = pv.z, q3 = pv.w;
-        float4 o;
-        o.x = (float)(q0 * fma(q1, E[0], fma(q2, E[1], q3 * E[2])));
-        o.y = (float)(q1 * fma(q2, E[3], fma(q3, E[4], -q0 * E[0])));
-        o.z = (float)(q2 * fma(q3, E[5], fma(-q0, E[1], -q1 * E[3])));
-        o.w = (float)(q3 * fma(-q0, E[2], fma(-q1, E[4], -q2 * E[5])));
-        if (!ok) o = make_float4(__int_as_float(0x7fffffff), __int_as_float(0x7fffffff),
-                                 __int_as_float(0x7fffffff), __int_as_float(0x7fffffff));
-        O4[r] = o;
-    }
-}
-
 }  // namespace mhc

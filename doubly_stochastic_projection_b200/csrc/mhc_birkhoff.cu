@@ -99,16 +99,16 @@ implicit_bwd_kernel(const float* logits, const float* P, const float* dP, float*
     pdl_wait();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
+        float p[16], g[16], out[16];
         if (kRecompute) {
-            float p[16], g[16], out[16];
             load16(logits + 16 * m, p);
             newton_project(p, kDefaultNewtonIters);
-            load16(dP + 16 * m, g);
-            implicit_vjp(p, g, out);
-            store16(dlogits + 16 * m, out);
         } else {
-            implicit_vjp_rows(P + 16 * m, dP + 16 * m, dlogits + 16 * m);
+            load16(P + 16 * m, p);
         }
+        load16(dP + 16 * m, g);
+        implicit_vjp(p, g, out);
+        store16(dlogits + 16 * m, out);
     }
 }
 
