@@ -121,10 +121,16 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# The sources the benchmark's two kernels (newton_fwd_kernel, implicit_bwd_kernel)
+# are compiled from; the committed DRAM-traffic capture is used only while
+# these are unchanged.
+TRAFFIC_SOURCES = ("birkhoff_math.cuh", "launch.h", "mhc_birkhoff.cu", "pdl.cuh")
+
+
 def csrc_hash():
     h = hashlib.sha256()
     d = os.path.join(ROOT, "doubly_stochastic_projection_b200", "csrc")
-    for name in sorted(os.listdir(d)):
+    for name in TRAFFIC_SOURCES:
         with open(os.path.join(d, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -780,51 +786,66 @@ def run_b200(args):
     api.birkhoff_fwd(A, "newton", out=P)
     polished = near_permutation_fraction(P)
 
-    # end to end through the C ABI with pinned host buffers: the native
-    # pipeline uploads, projects, differentiates and downloads in pieces
+    # end to end through the C ABI with pinned host buffers, copies or PCIe
+    # traffic inside the timed region, two ways: the kernels reading and
+    # writing the pinned buffers directly (zero-copy), and the copy pipeline
+    # (pieces uploaded, computed and downloaded on overlapping streams)
     A_h = A.cpu().pin_memory()
     G_h = G.cpu().pin_memory()
     P_h = torch.empty_like(A_h).pin_memory()
     dl_h = torch.empty_like(A_h).pin_memory()
     work = [torch.empty_like(A) for _ in range(4)]
     pieces = args.e2e_pieces
-
-    def e2e_step():
-        api.birkhoff_fwd_bwd_host(A_h, G_h, P_h, dl_h, work, pieces)
-
+    e2e_paths = {
+        "mapped": lambda: api.birkhoff_fwd_bwd_mapped(A_h, G_h, P_h, dl_h, work[2]),
+        "pipelined": lambda: api.birkhoff_fwd_bwd_host(A_h, G_h, P_h, dl_h, work, pieces),
+    }
     e2e_steps = max(3, min(K, 50))
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize()
-    tot = 0.0
-    for i in range(e2e_steps):
-        f0 = torch.cuda.Event(enable_timing=True)
-        f1 = torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        e2e_step()
-        f1.record(stream)
-        f1.synchronize()
-        tot += f0.elapsed_time(f1) * 1e-3
-    t_e2e = max_over_ranks(tot / e2e_steps, pg, dev)
-    # one more step with the device staging poisoned first: a kernel that read
-    # its inputs before their upload landed would leave NaN in the host results
-    for w in work:
-        w.fill_(float("nan"))
-    P_h.zero_()
-    dl_h.zero_()
-    e2e_step()
-    torch.cuda.synchronize()
+    e2e_t = {}
+    for name, fn in e2e_paths.items():
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for i in range(e2e_steps):
+            f0 = torch.cuda.Event(enable_timing=True)
+            f1 = torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            fn()
+            f1.record(stream)
+            f1.synchronize()
+            tot += f0.elapsed_time(f1) * 1e-3
+        e2e_t[name] = max_over_ranks(tot / e2e_steps, pg, dev)
+    # one more step of each with the device buffers poisoned first and the host
+    # outputs zeroed: a kernel that read its inputs before they arrived would
+    # leave NaN in the host results
     api.birkhoff_fwd(A, "newton", out=P)
     api.birkhoff_bwd(G, P=P, out=dl)
-    matches = bool(torch.equal(dl_h, dl.cpu()) and torch.equal(P_h, P.cpu()))
+    matches = {}
+    for name, fn in e2e_paths.items():
+        for w in work:
+            w.fill_(float("nan"))
+        P_h.zero_()
+        dl_h.zero_()
+        fn()
+        torch.cuda.synchronize()
+        # (the zero-copy kernels inline the same solver into other kernels:
+        # equal up to rounding)
+        matches[name] = bool((P_h - P.cpu()).abs().max().item() <= 2e-6 and
+                             (dl_h - dl.cpu()).abs().max().item() <= 1e-5 * dl.abs().max().item())
     nbytes = 2 * A.numel() * 4
+    t_e2e = e2e_t["mapped"]
     e2e = {"value": world * N_MATS / t_e2e, "unit": UNIT, "h2d_bytes_per_step": nbytes,
            "d2h_bytes_per_step": nbytes, "ms_per_step": t_e2e * 1e3,
            "h2d_gbs": nbytes / t_e2e / 1e9, "d2h_gbs": nbytes / t_e2e / 1e9,
-           "path": "mhc_birkhoff_fwd_bwd_host (C ABI): pinned host -> device copies, Newton fwd, implicit bwd, "
-                   "device -> host copies of P and dlogits, in %d pieces on two copy streams and the "
-                   "launching stream" % pieces,
-           "matches_device_run": matches}
+           "path": "mhc_birkhoff_fwd_bwd_mapped (C ABI): the Newton forward reads the logits from pinned host "
+                   "memory and writes P to it (and to device memory), the implicit backward reads dP from and "
+                   "writes dlogits to pinned host memory, over PCIe, inside the timed region",
+           "matches_device_run": matches["mapped"],
+           "pipelined": {"value": world * N_MATS / e2e_t["pipelined"], "ms_per_step": e2e_t["pipelined"] * 1e3,
+                         "path": "mhc_birkhoff_fwd_bwd_host: copies in %d pieces on two copy streams, kernels on "
+                                 "the launching stream" % pieces,
+                         "matches_device_run": matches["pipelined"]}}
 
     # dominant kernel and its roofline
     mhz = clocks.max_mhz or 1965

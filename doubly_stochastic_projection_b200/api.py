@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
                 "mhc_proj_mix_fwd": [p, p, p, p, p, p, i64, i64, i32, p],
                 "mhc_proj_mix_bwd": [p, p, p, p, p, p, p, p, p, i64, i64, p],
                 "mhc_birkhoff_fwd_bwd_host": [p, p, p, p, p, p, p, p, i64, i32, p],
+                "mhc_birkhoff_fwd_bwd_mapped": [p, p, p, p, p, i64, p],
             }
             for name, args in sig.items():
                 f = getattr(L, name)
@@ -212,6 +213,29 @@ def birkhoff_fwd_bwd_host(logits_h, dP_h, P_h, dlogits_h, work, pieces: int = 4)
     n = _n_mats(logits_h)
     _check(lib().mhc_birkhoff_fwd_bwd_host(_ptr(logits_h), _ptr(dP_h), _ptr(P_h), _ptr(dlogits_h),
                                            *[_ptr(t) for t in work], n, int(pieces), _stream(work[0])))
+
+
+def _host_batch(logits_h, dP_h, P_h, dlogits_h):
+    for name, t in (("logits_h", logits_h), ("dP_h", dP_h), ("P_h", P_h), ("dlogits_h", dlogits_h)):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous float32 CPU tensor" % name)
+        if not t.is_pinned():
+            raise ValueError("%s must be in pinned (page-locked) host memory" % name)
+        if t.shape != logits_h.shape:
+            raise ValueError("%s must have shape %s" % (name, tuple(logits_h.shape)))
+    return _n_mats(logits_h)
+
+
+def birkhoff_fwd_bwd_mapped(logits_h, dP_h, P_h, dlogits_h, P_d):
+    """Newton forward + implicit backward of a batch in pinned host memory with
+    no copies: the kernels read and write the host buffers over PCIe
+    (mhc_birkhoff_fwd_bwd_mapped).  ``P_d`` is a device tensor of the same
+    shape for the forward's P.  Asynchronous on the current stream of P_d's
+    device; synchronise it before reading the host outputs."""
+    n = _host_batch(logits_h, dP_h, P_h, dlogits_h)
+    _need(P_d, "P_d", torch.float32, logits_h.shape)
+    _check(lib().mhc_birkhoff_fwd_bwd_mapped(_ptr(logits_h), _ptr(dP_h), _ptr(P_h), _ptr(dlogits_h), _ptr(P_d), n,
+                                             _stream(P_d)))
 
 
 def _square(t, name):

@@ -16,6 +16,7 @@
 #include "birkhoff_math.cuh"
 #include "launch.h"
 #include "mhc_birkhoff.h"
+#include "pdl.cuh"
 
 namespace {
 
@@ -104,4 +105,109 @@ extern "C" int mhc_birkhoff_fwd_bwd_host(const float* logits_h, const float* dP_
     if (e == cudaSuccess) e = cudaEventRecord(p.done, p.out);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(s, p.done, 0);
     return e == cudaSuccess ? MHC_OK : MHC_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Zero-copy variant: the kernels read the pinned host inputs and write the
+// host outputs themselves, over PCIe, through the buffers' mapped device
+// addresses.  A forward reads logits from the host while it writes P to the
+// host (both directions of the link at once), and the backward does the same
+// with dP and dlogits; no copy engine and no pieces are involved.  The
+// forward keeps a device copy of P for the backward: the one buffer of device
+// memory the call needs.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kMirrorThreads = 128;
+
+// A matrix read with plain (coherent) loads: host memory is not read through
+// the read-only cache path.
+__device__ __forceinline__ void load16_host(const float* p, float (&a)[16])
+{
+    const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const float4 v = q[r];
+        a[4 * r + 0] = v.x;
+        a[4 * r + 1] = v.y;
+        a[4 * r + 2] = v.z;
+        a[4 * r + 3] = v.w;
+    }
+}
+
+// Newton forward (MHC_NEWTON) of logits in host memory that stores P twice:
+// into P (device memory, read by the backward) and into P_mirror (the
+// caller's host buffer).
+__global__ void __launch_bounds__(kMirrorThreads)
+newton_fwd_mirror_kernel(const float* logits, float* P, float* P_mirror, int64_t n, int maxit)
+{
+    mhc::pdl_wait();
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
+        float a[16];
+        load16_host(logits + 16 * m, a);
+        mhc::newton_project(a, maxit);
+        mhc::store16(P + 16 * m, a);
+        mhc::store16(P_mirror + 16 * m, a);
+    }
+}
+
+// Implicit backward with P in device memory and dP, dlogits in host memory.
+__global__ void __launch_bounds__(kMirrorThreads)
+implicit_bwd_host_kernel(const float* P, const float* dP, float* dlogits, int64_t n)
+{
+    mhc::pdl_wait();
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
+        float p[16], g[16], out[16];
+        mhc::load16(P + 16 * m, p);
+        load16_host(dP + 16 * m, g);
+        mhc::implicit_vjp(p, g, out);
+        mhc::store16(dlogits + 16 * m, out);
+    }
+}
+
+bool mapped(const void* host, void** dev)
+{
+    if (cudaHostGetDevicePointer(dev, const_cast<void*>(host), 0) != cudaSuccess || *dev == nullptr) {
+        cudaGetLastError();
+        return false;
+    }
+    return true;
+}
+
+}  // namespace
+
+namespace mhc {
+
+int fwd_bwd_mapped(const float* logits_h, const float* dP_h, float* P_h, float* dlogits_h, float* P_d, int64_t n_mats,
+                   cudaStream_t s)
+{
+    void *lg = nullptr, *dp = nullptr, *ph = nullptr, *dl = nullptr;
+    if (!mapped(logits_h, &lg) || !mapped(dP_h, &dp) || !mapped(P_h, &ph) || !mapped(dlogits_h, &dl))
+        return MHC_ERR_ARG;
+    const int64_t need = (n_mats + kMirrorThreads - 1) / kMirrorThreads;
+    const int fb = persistent_grid((const void*)newton_fwd_mirror_kernel, kMirrorThreads, 0, need);
+    cudaError_t e = launch_pdl(newton_fwd_mirror_kernel, fb, kMirrorThreads, 0, s, (const float*)lg, P_d,
+                               (float*)ph, n_mats, kDefaultNewtonIters);
+    const int bb = persistent_grid((const void*)implicit_bwd_host_kernel, kMirrorThreads, 0, need);
+    if (e == cudaSuccess)
+        e = launch_pdl(implicit_bwd_host_kernel, bb, kMirrorThreads, 0, s, (const float*)P_d, (const float*)dp,
+                       (float*)dl, n_mats);
+    return e == cudaSuccess ? MHC_OK : MHC_ERR_CUDA;
+}
+
+}  // namespace mhc
+
+extern "C" int mhc_birkhoff_fwd_bwd_mapped(const float* logits_h, const float* dP_h, float* P_h, float* dlogits_h,
+                                           float* P_d, int64_t n_mats, void* stream)
+{
+    if (n_mats < 0 || n_mats > (int64_t(1) << 36)) return MHC_ERR_SIZE;
+    if (n_mats == 0) return MHC_OK;
+    if (!logits_h || !dP_h || !P_h || !dlogits_h || !P_d) return MHC_ERR_NULL;
+    if (misaligned(logits_h) || misaligned(dP_h) || misaligned(P_h) || misaligned(dlogits_h) || misaligned(P_d))
+        return MHC_ERR_ALIGN;
+    if (!pinned_host(logits_h) || !pinned_host(dP_h) || !pinned_host(P_h) || !pinned_host(dlogits_h))
+        return MHC_ERR_ARG;
+    return mhc::fwd_bwd_mapped(logits_h, dP_h, P_h, dlogits_h, P_d, n_mats, static_cast<cudaStream_t>(stream));
 }

@@ -395,6 +395,29 @@ MHC_API int mhc_birkhoff_fwd_bwd_host(const float *logits_h, const float *dP_h, 
                                       float *logits_d, float *dP_d, float *P_d, float *dlogits_d,
                                       int64_t n_mats, int pieces, void *stream);
 
+/*
+ * mhc_birkhoff_fwd_bwd_mapped -- the same computation as
+ * mhc_birkhoff_fwd_bwd_host, with no copies: the kernels read logits and dP
+ * from the pinned host buffers and write P and dlogits into them directly,
+ * over PCIe, through the buffers' mapped device addresses (zero-copy).  The
+ * forward reads from the host while it writes to it, so both directions of
+ * the link are busy at once; so is the backward.  P_d is device memory for
+ * the forward's P, which the backward reads.
+ *
+ *   logits_h, dP_h    [n_mats][4][4] float, PINNED host memory, read.
+ *   P_h, dlogits_h    [n_mats][4][4] float, PINNED host memory, written.
+ *   P_d               [n_mats][4][4] float, device, scratch (overwritten).
+ *   Every pointer must be 16-byte aligned.  A host buffer that is not
+ *   page-locked, or that CUDA cannot map into the device's address space,
+ *   returns MHC_ERR_ARG.
+ *
+ * Ordering: as any call on `stream`; synchronising `stream` makes P_h and
+ * dlogits_h readable.  The host buffers must not be touched by the host
+ * while the call runs.
+ */
+MHC_API int mhc_birkhoff_fwd_bwd_mapped(const float *logits_h, const float *dP_h, float *P_h, float *dlogits_h,
+                                        float *P_d, int64_t n_mats, void *stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 MHC_API const char *mhc_status_string(int status);
 

@@ -112,6 +112,11 @@ def test_validation_of_the_remaining_entry_points(L):
     assert L.mhc_birkhoff_fwd_bwd_host(*[None] * 8, 0, 4, None) == 0             # nothing to do
     assert L.mhc_birkhoff_fwd_bwd_host(None, *[fake] * 7, 10, 4, None) == 1
     assert L.mhc_birkhoff_fwd_bwd_host(*[fake] * 7, fake + 4, 10, 4, None) == 2
+    L.mhc_birkhoff_fwd_bwd_mapped.argtypes = [p, p, p, p, p, i64, p]
+    assert L.mhc_birkhoff_fwd_bwd_mapped(*[fake] * 5, -1, None) == 3
+    assert L.mhc_birkhoff_fwd_bwd_mapped(*[None] * 5, 0, None) == 0
+    assert L.mhc_birkhoff_fwd_bwd_mapped(fake, fake, fake, fake, None, 10, None) == 1
+    assert L.mhc_birkhoff_fwd_bwd_mapped(fake, fake, fake + 8, fake, fake, 10, None) == 2
     L.mhc_residual_mix_bwd.argtypes = [p, p, p, p, p, p, p, p, p, p, i64, i64, p]
     assert L.mhc_residual_mix_bwd(fake, fake, fake, fake, fake, fake, None, None, fake, None, 1 << 36, 1 << 24,
                                   None) == 3                                    # T * 4 * C above 2^40
