@@ -238,6 +238,20 @@ def birkhoff_fwd_bwd_mapped(logits_h, dP_h, P_h, dlogits_h, P_d):
                                              _stream(P_d)))
 
 
+def birkhoff_fwd_bwd_mapped_static(logits_h, dP_h, P_h, dlogits_h):
+    """birkhoff_fwd_bwd_mapped for callers that cannot allocate device memory
+    (mhc_birkhoff_fwd_bwd_mapped_static): the forward's P goes to a fixed
+    array inside the library, so the call allocates nothing.  At most
+    MHC_NOALLOC_MAX_MATS (262144) matrices a call.  Runs on the current CUDA
+    device and its current stream; calls that can overlap on the GPU share the
+    array and race, so keep them on one stream."""
+    n = _host_batch(logits_h, dP_h, P_h, dlogits_h)
+    f = lib().mhc_birkhoff_fwd_bwd_mapped_static
+    f.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int64, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    _check(f(_ptr(logits_h), _ptr(dP_h), _ptr(P_h), _ptr(dlogits_h), n, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)))
+
+
 def _square(t, name):
     if t.dim() < 2 or t.shape[-1] != t.shape[-2]:
         raise ValueError("%s must be [..., n, n], got %s" % (name, tuple(t.shape)))

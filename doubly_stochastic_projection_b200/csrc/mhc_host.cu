@@ -280,3 +280,63 @@ extern "C" int mhc_birkhoff_fwd_bwd_mapped(const float* logits_h, const float* d
         return MHC_ERR_ARG;
     return mhc::fwd_bwd_mapped(logits_h, dP_h, P_h, dlogits_h, P_d, n_mats, static_cast<cudaStream_t>(stream));
 }
+
+// ---------------------------------------------------------------------------
+// The zero-copy path for callers that cannot allocate device memory.
+//
+// Some callers may not call cudaMalloc, or any allocator, while they run: a
+// plugin inside a host application that owns all device memory through its
+// own pool and hands its plugins none; a real-time loop, where cudaMalloc's
+// device-wide synchronisation would stall every other stream; a process that
+// must not fail for lack of memory in the middle of a step.  For them the
+// forward's P, the only device memory the zero-copy path needs beyond the
+// caller's host buffers, lives in the file-scope array below.  The CUDA
+// runtime reserves it on each GPU where this library's code is loaded and
+// keeps it there until the process exits: MHC_NOALLOC_MAX_MATS matrices,
+// 16 MiB.  Every call on a device shares it.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) float g_noalloc_P[(size_t)MHC_NOALLOC_MAX_MATS * 16];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_P on device `dev`, which must be current.  In
+// host code the name g_noalloc_P only stands for the array; its address on a
+// device comes from cudaGetSymbolAddress, looked up on the first call on that
+// device and kept.
+float* noalloc_scratch(int dev)
+{
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_P) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        g_noalloc_ptr[dev] = static_cast<float*>(p);
+    }
+    return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" int mhc_birkhoff_fwd_bwd_mapped_static(const float* logits_h, const float* dP_h, float* P_h,
+                                                  float* dlogits_h, int64_t n_mats, void* stream)
+{
+    if (n_mats < 0 || n_mats > MHC_NOALLOC_MAX_MATS) return MHC_ERR_SIZE;
+    if (n_mats == 0) return MHC_OK;
+    if (!logits_h || !dP_h || !P_h || !dlogits_h) return MHC_ERR_NULL;
+    if (misaligned(logits_h) || misaligned(dP_h) || misaligned(P_h) || misaligned(dlogits_h)) return MHC_ERR_ALIGN;
+    if (!pinned_host(logits_h) || !pinned_host(dP_h) || !pinned_host(P_h) || !pinned_host(dlogits_h))
+        return MHC_ERR_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MHC_ERR_CUDA;
+    float* P_d = noalloc_scratch(dev);
+    if (P_d == nullptr) return MHC_ERR_CUDA;
+    // nothing in the array has to start at zero: the forward writes every
+    // matrix of P that the backward then reads, so what an earlier call left
+    // there is never read
+    return mhc::fwd_bwd_mapped(logits_h, dP_h, P_h, dlogits_h, P_d, n_mats, static_cast<cudaStream_t>(stream));
+}

@@ -418,6 +418,46 @@ MHC_API int mhc_birkhoff_fwd_bwd_host(const float *logits_h, const float *dP_h, 
 MHC_API int mhc_birkhoff_fwd_bwd_mapped(const float *logits_h, const float *dP_h, float *P_h, float *dlogits_h,
                                         float *P_d, int64_t n_mats, void *stream);
 
+/* Largest batch mhc_birkhoff_fwd_bwd_mapped_static accepts: the number of
+ * 4x4 float matrices its fixed device array holds (16 MiB). */
+#define MHC_NOALLOC_MAX_MATS 262144
+
+/*
+ * mhc_birkhoff_fwd_bwd_mapped_static -- mhc_birkhoff_fwd_bwd_mapped without
+ * the caller's device buffer: the call allocates nothing.  The paper has no
+ * counterpart; this is a deployment variant.
+ *
+ * It is for callers that cannot allocate device memory while they run: a
+ * plugin whose host application owns all device memory through its own pool,
+ * a real-time loop where cudaMalloc's device-wide synchronisation would stall
+ * other streams, a process that must not fail for lack of memory in the
+ * middle of a step.  The forward's P goes to a fixed array inside the library
+ * instead (MHC_NOALLOC_MAX_MATS matrices, 16 MiB), which the CUDA runtime
+ * reserves on every GPU where the library's code is loaded and keeps there
+ * until the process exits.  The call makes no cudaMalloc, cudaFree or other
+ * allocating call.
+ *
+ *   logits_h, dP_h    [n_mats][4][4] float, PINNED host memory, read.
+ *   P_h, dlogits_h    [n_mats][4][4] float, PINNED host memory, written.
+ *   n_mats            0 .. MHC_NOALLOC_MAX_MATS; a larger (or negative)
+ *                     n_mats returns MHC_ERR_SIZE and enqueues nothing.
+ *   Alignment, pinning and the other errors: as mhc_birkhoff_fwd_bwd_mapped.
+ *   The call runs on the current device, on `stream`.
+ *
+ * Set-up: the first call on a device looks up the array's address on that
+ * device (cudaGetSymbolAddress) and keeps it; make that first call before
+ * any stream capture on the device.
+ *
+ * Sharing: every call on a device uses the same array, and the array keeps
+ * what the last call wrote.  Nothing in it needs to start at zero (the
+ * forward writes every matrix the backward reads).  Calls that can overlap on
+ * the GPU (on different streams, or from several host threads without an
+ * ordering between their streams) race on the array and give wrong results:
+ * issue them on one stream, or order them with events.
+ */
+MHC_API int mhc_birkhoff_fwd_bwd_mapped_static(const float *logits_h, const float *dP_h, float *P_h,
+                                               float *dlogits_h, int64_t n_mats, void *stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 MHC_API const char *mhc_status_string(int status);
 

@@ -122,6 +122,19 @@ def test_validation_of_the_remaining_entry_points(L):
                                   None) == 3                                    # T * 4 * C above 2^40
 
 
+def test_validation_of_the_no_alloc_entry_point(L):
+    p, i64 = ctypes.c_void_p, ctypes.c_int64
+    fake = 1 << 20  # never dereferenced: every call below returns before any CUDA call
+    cap = int(re.search(r"#define\s+MHC_NOALLOC_MAX_MATS\s+(\d+)", open(HEADER).read()).group(1))
+    f = L.mhc_birkhoff_fwd_bwd_mapped_static
+    f.argtypes = [p, p, p, p, i64, p]
+    assert f(*[fake] * 4, cap + 1, None) == 3                                    # beyond the fixed array
+    assert f(*[fake] * 4, -1, None) == 3
+    assert f(*[None] * 4, 0, None) == 0
+    assert f(fake, fake, None, fake, 10, None) == 1
+    assert f(fake, fake, fake, fake + 8, 10, None) == 2
+
+
 def test_header_is_plain_c(tmp_path):
     # the boundary is usable from C: the header compiles as strict C99 and a C
     # program links the library and runs a host-only call
