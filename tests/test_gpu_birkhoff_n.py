@@ -88,3 +88,35 @@ def test_projection_n_many_tiles_per_cta(orc, n):
     dref = orc.implicit_bwd(row_normalised(P[idx]), G[idx].astype(np.float64))
     rel, _ = per_matrix_rel_err(dl[idx].reshape(len(idx), -1), dref.reshape(len(idx), -1))
     assert rel.max() <= GRAD_REL_TOL, rel.max()
+
+
+@pytest.mark.parametrize("n", [3, 5, 8])
+@pytest.mark.parametrize("kind", ["normal10", "near_permutation"])
+def test_implicit_bwd_n_on_peaked_matrices(orc, n, kind):
+    # rows close to one-hot, where a weighted-mean form of the softmax Jacobian
+    # would cancel: the backward at the kernel's own P against the oracle's
+    count = 2048 + 13
+    rng = np.random.default_rng(500 + n)
+    if kind == "normal10":
+        A = (rng.standard_normal((count, n, n)) * 10.0).astype(np.float32)
+    else:
+        perm = np.argsort(rng.random((count, n)), axis=1)
+        A = rng.standard_normal((count, n, n)).astype(np.float32)
+        A[np.arange(count)[:, None], np.arange(n)[None, :], perm] += 8.0
+    G = _logits(count, n, 1.0, 600 + n)
+    P_g = api.birkhoff_fwd_n(to_gpu(A), "newton")
+    P = to_np64(P_g)
+    assert np.isfinite(P).all() and P.min() >= 0
+    assert np.abs(P.sum(-1) - 1).max() <= SUM_TOL and np.abs(P.sum(-2) - 1).max() <= SUM_TOL
+    # both sides take the same input, a point of the polytope to fp32
+    # rounding: the oracle's P (converged to 1e-12), rows renormalised, in
+    # fp32.  The forward's own P is off the polytope by up to its 1e-6
+    # stopping tolerance, and there two exact forms of the backward (the
+    # kernel's and the oracle's) part by more than the bar on ill-conditioned
+    # matrices: that gap measures the input, not the backward.
+    ref_P = orc.newton(A.astype(np.float64), tol=1e-12, max_iter=200)
+    P_in = row_normalised(ref_P).astype(np.float32)
+    dl = to_np64(api.birkhoff_bwd_n(to_gpu(G), to_gpu(P_in)))
+    dref = orc.implicit_bwd(row_normalised(P_in), G.astype(np.float64))
+    rel, _ = per_matrix_rel_err(dl.reshape(count, -1), dref.reshape(count, -1))
+    assert rel.max() <= GRAD_REL_TOL, (n, kind, rel.max())
