@@ -80,22 +80,36 @@ __device__ __forceinline__ constexpr int edge(int j, int k)
 // by eliminating columns 0..N-3 in turn (Kron reduction: each elimination
 // only adds positive weights, so no pivot is formed by cancellation).  W and
 // rhs are overwritten.  T is float or double.
+// Reciprocal of an elimination pivot: fp32 (the forward's Newton direction)
+// takes the 1-ulp MUFU reciprocal, fp64 (the backward) the exact one.
+template <typename T>
+__device__ __forceinline__ T pivot_rcp(T a)
+{
+    return T(1) / a;
+}
+
+template <>
+__device__ __forceinline__ float pivot_rcp<float>(float a)
+{
+    return rcp_approx(a);
+}
+
 template <int N, typename T>
 __device__ __forceinline__ bool grounded_laplacian_solve(T (&W)[N * (N - 1) / 2], T (&rhs)[N], T mu, T (&x)[N])
 {
     static_assert(N >= 2, "needs a free column");
 #pragma unroll
     for (int j = 0; j + 1 < N; ++j) W[edge<N>(j, N - 1)] += mu;
-    T piv[N];
+    T ipiv[N];  // reciprocals of the pivots, reused by the back substitution
     bool ok = true;
 #pragma unroll
     for (int p = 0; p + 1 < N; ++p) {
         T a = T(0);
 #pragma unroll
         for (int k = p + 1; k < N; ++k) a += W[edge<N>(p, k)];
-        piv[p] = a;
         ok = ok && (a > T(0));
-        const T ia = T(1) / a;
+        const T ia = pivot_rcp<T>(a);
+        ipiv[p] = ia;
 #pragma unroll
         for (int i = p + 1; i + 1 < N; ++i) {
             rhs[i] += W[edge<N>(p, i)] * rhs[p] * ia;
@@ -108,7 +122,7 @@ __device__ __forceinline__ bool grounded_laplacian_solve(T (&W)[N * (N - 1) / 2]
         T s = rhs[p];
 #pragma unroll
         for (int k = p + 1; k + 1 < N; ++k) s += W[edge<N>(p, k)] * x[k];
-        x[p] = s / piv[p];
+        x[p] = s * ipiv[p];
     }
     x[N - 1] = T(0);
     T tot = T(0);
