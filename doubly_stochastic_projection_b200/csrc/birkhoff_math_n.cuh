@@ -112,9 +112,10 @@ __device__ __forceinline__ bool grounded_laplacian_solve(T (&W)[N * (N - 1) / 2]
         ipiv[p] = ia;
 #pragma unroll
         for (int i = p + 1; i + 1 < N; ++i) {
-            rhs[i] += W[edge<N>(p, i)] * rhs[p] * ia;
+            const T t = W[edge<N>(p, i)] * ia;  // one product a row, then one fma an update
+            rhs[i] = fma(t, rhs[p], rhs[i]);
 #pragma unroll
-            for (int k = i + 1; k < N; ++k) W[edge<N>(i, k)] += W[edge<N>(p, i)] * W[edge<N>(p, k)] * ia;
+            for (int k = i + 1; k < N; ++k) W[edge<N>(i, k)] = fma(t, W[edge<N>(p, k)], W[edge<N>(i, k)]);
         }
     }
 #pragma unroll
@@ -253,9 +254,13 @@ __device__ __forceinline__ int newton_project_n(float (&a)[N * N], int maxit)
             float t = 1.0f;
             ok = false;
             for (int h = 0; h < kMaxHalvings && slope < 0.0f; ++h) {
-                float lg = 0.0f;
+                // one logarithm of the product of the row sums: with steps
+                // capped at kStepCap every s_r lies in [e^-4, e^4], so the
+                // product of N <= 8 of them stays within [e^-32, e^32]
+                float prod = s[0];
 #pragma unroll
-                for (int r = 0; r < N; ++r) lg += __logf(s[r]);
+                for (int r = 1; r < N; ++r) prod *= s[r];
+                const float lg = __logf(prod);
                 if (lg - t * dsum <= kArmijo * t * slope) {
                     ok = true;
                     break;
