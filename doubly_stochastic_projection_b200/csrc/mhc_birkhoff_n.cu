@@ -7,9 +7,10 @@
 // matrix occupies an odd number of words in shared memory, so the threads of a
 // warp reading the same entry of their matrices hit 32 different banks.
 // Measured on B200 at 1M matrices, n = 8: Newton 1.29 -> 3.42 G/s, implicit
-// backward 0.82 -> 2.82 G/s.  For n = 2, 3 the two barriers per tile cost more
-// than the coalescing gains (Sinkhorn and the backward 5-18% slower), and
-// those sizes keep direct per-thread loads.
+// backward 0.82 -> 2.82 G/s.  n = 3 is staged too since the tiles are copied
+// with cp.async (backward 3965 -> 4872 GB/s, forward +3%, at 7.5M matrices);
+// with plain loads and stores it had been 5-18% slower than direct loads.
+// n = 2 (closed forms, 16-byte matrices) keeps direct per-thread loads.
 #include "birkhoff_math_n.cuh"
 #include "launch.h"
 #include "pdl.cuh"
@@ -21,7 +22,7 @@ namespace {
 constexpr int kThreadsN = 128;
 
 template <int N>
-constexpr bool kTiled = N >= 5;
+constexpr bool kTiled = N >= 3;
 
 template <int N>
 __device__ __forceinline__ void load_n(const float* p, float (&a)[N * N])
