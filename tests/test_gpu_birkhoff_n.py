@@ -120,3 +120,20 @@ def test_implicit_bwd_n_on_peaked_matrices(orc, n, kind):
     dref = orc.implicit_bwd(row_normalised(P_in), G.astype(np.float64))
     rel, _ = per_matrix_rel_err(dl.reshape(count, -1), dref.reshape(count, -1))
     assert rel.max() <= GRAD_REL_TOL, (n, kind, rel.max())
+
+
+@pytest.mark.parametrize("n", [2, 3, 8])
+def test_n_in_place(n):
+    # P may equal logits and dlogits may equal dP (each matrix, or each staged
+    # tile, is read whole before it is written): in place gives the same bits
+    count = 3 * 128 + 5
+    A = to_gpu(_logits(count, n, 3.0, 700 + n))
+    G = to_gpu(_logits(count, n, 1.0, 800 + n))
+    P_ref = api.birkhoff_fwd_n(A.clone(), "newton")
+    dl_ref = api.birkhoff_bwd_n(G.clone(), P_ref)
+    A_in = A.clone()
+    P_in = api.birkhoff_fwd_n(A_in, "newton", out=A_in)
+    assert P_in.data_ptr() == A_in.data_ptr() and torch.equal(P_in, P_ref)
+    G_in = G.clone()
+    dl_in = api.birkhoff_bwd_n(G_in, P_ref, out=G_in)
+    assert dl_in.data_ptr() == G_in.data_ptr() and torch.equal(dl_in, dl_ref)
