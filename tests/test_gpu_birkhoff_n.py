@@ -137,3 +137,22 @@ def test_n_in_place(n):
     G_in = G.clone()
     dl_in = api.birkhoff_bwd_n(G_in, P_ref, out=G_in)
     assert dl_in.data_ptr() == G_in.data_ptr() and torch.equal(dl_in, dl_ref)
+
+
+@pytest.mark.parametrize("n", [2, 3, 5, 8])
+def test_n_degenerate_inputs(orc, n):
+    # constant and additive logits project to J / n exactly; scaled identity and
+    # permutation logits to matrices close to them; all against the oracle
+    rng = np.random.default_rng(900 + n)
+    perm = np.eye(n)[rng.permutation(n)]
+    cases = [np.zeros((n, n)), np.full((n, n), 1e4),
+             rng.standard_normal((n, 1)) * 5 + rng.standard_normal((1, n)) * 5,
+             30.0 * np.eye(n), 40.0 * perm, -30.0 * np.eye(n)]
+    A = np.stack(cases).astype(np.float32)
+    P = to_np64(api.birkhoff_fwd_n(to_gpu(A), "newton"))
+    ref = orc.newton(A.astype(np.float64), tol=1e-12, max_iter=200)
+    assert np.isfinite(P).all()
+    assert np.abs(P - ref).max() <= P_ABS_TOL
+    for k in (0, 1, 2):
+        assert np.abs(P[k] - 1.0 / n).max() <= 1e-6, k
+    assert np.abs(P.sum(-1) - 1).max() <= SUM_TOL and np.abs(P.sum(-2) - 1).max() <= SUM_TOL
