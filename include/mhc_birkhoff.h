@@ -387,7 +387,9 @@ MHC_API int mhc_composite_gain(const float *P_layers, float *M, float *gain_rows
  * and work enqueued on `stream` afterwards sees every output written (host
  * outputs included, so synchronising `stream` makes P_h and dlogits_h
  * readable).  The library creates its two copy streams and their events once
- * per device, on the first call, and keeps them until the process exits.
+ * per device, on the first call, and keeps them until the process exits; they
+ * belong to the device's context at that time, so a process that resets the
+ * device (cudaDeviceReset) must not call this entry point on it afterwards.
  * Calls from several host threads are serialised internally while they
  * enqueue.
  */
@@ -446,7 +448,9 @@ MHC_API int mhc_birkhoff_fwd_bwd_mapped(const float *logits_h, const float *dP_h
  *
  * Set-up: the first call on a device looks up the array's address on that
  * device (cudaGetSymbolAddress) and keeps it; make that first call before
- * any stream capture on the device.
+ * any stream capture on the device.  The kept address belongs to the device's
+ * context at that time: a process that resets the device (cudaDeviceReset)
+ * must not call this entry point on it afterwards.
  *
  * Sharing: every call on a device uses the same array, and the array keeps
  * what the last call wrote.  Nothing in it needs to start at zero (the
