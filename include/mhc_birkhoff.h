@@ -366,7 +366,9 @@ MHC_API int mhc_composite_gain(const float *P_layers, float *M, float *gain_rows
 /*
  * mhc_birkhoff_fwd_bwd_host -- the projection's forward and implicit backward
  * (as mhc_birkhoff_fwd with MHC_NEWTON followed by mhc_birkhoff_bwd with the
- * saved P) for a batch held in pinned host memory, copies included.  The
+ * saved P: [BA] §2.1 and §2.2) for a batch held in pinned host memory, copies
+ * included.  The pages describe no transfer scheme; this one is the
+ * library's own.  The
  * batch is cut into `pieces` contiguous pieces; the upload of a piece, the
  * two kernels of the previous piece and the download of the one before run
  * concurrently (PCIe carries both directions at once), on two copy streams
