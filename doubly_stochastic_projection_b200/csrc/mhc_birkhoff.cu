@@ -26,11 +26,13 @@ namespace {
 
 constexpr int kProjThreads = 256;
 // Batches that fit in about two waves of 256-thread CTAs are launched with
-// 128-thread CTAs instead: twice as many CTAs spread the batch (and its mix
-// of easy and hard matrices) more evenly over the 148 SMs.  Measured on B200:
-// 131072 matrices, Newton 18.4 -> 16.4 us, backward 12.3 -> 11.2 us; at 16M
-// matrices 256-thread CTAs are 1-2% faster.
-constexpr int kProjThreadsSmall = 128;
+// 64-thread CTAs instead: more, smaller CTAs spread the batch (and its mix of
+// easy and hard matrices) more evenly over the 148 SMs.  Measured on B200 at
+// 131072 matrices: Newton 18.4 us with 256-thread CTAs, 16.4 with 128 (one at
+// a time between L2 flushes); back to back, 12.08 us with 128 against 11.90
+// with 64 and 12.01 with 32, backward 6.45 against 6.35.  At 16M matrices
+// 256-thread CTAs are 1-2% faster.
+constexpr int kProjThreadsSmall = 64;
 
 __global__ void __launch_bounds__(kProjThreads)
 sinkhorn_fwd_kernel(const float* logits, float* P, int64_t n, int iters)
