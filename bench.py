@@ -111,14 +111,22 @@ def headline_config(world):
 # ----------------------------------------------------------------- helpers
 
 
-def measured_peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+def measured_peaks(path=None):
+    """HBM copy bandwidth (GB/s) from MEASURED_PEAKS.json and its source, or
+    the fallback figure.  The entry may be a number or an object holding one
+    (under "value", "gbs" or "burst")."""
+    path = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
-            d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
+            v = json.load(f)["hbm_gbs"]
+        if isinstance(v, dict):
+            v = next(v[k] for k in ("value", "gbs", "burst") if k in v)
+        v = float(v)
+        if v > 0:
+            return v, "measured"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
+        pass
+    return FALLBACK_HBM_GBS, "fallback"
 
 
 # The sources the benchmark's two kernels (newton_fwd_kernel, implicit_bwd_kernel)

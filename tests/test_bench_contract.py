@@ -66,3 +66,17 @@ def test_product_arm_has_no_cpu_fallback():
                         "--no-cpu-baseline"], cwd=ROOT, capture_output=True, text=True, timeout=300)
     assert r.returncode != 0
     assert not _json_lines(r.stdout)
+
+
+def test_measured_peaks_reader(tmp_path):
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    import bench
+    f = tmp_path / "peaks.json"
+    f.write_text(json.dumps({"hbm_gbs": 6542.7, "bf16_tflops": 1590}))
+    assert bench.measured_peaks(str(f)) == (6542.7, "measured")
+    f.write_text(json.dumps({"hbm_gbs": {"value": 6500.0, "unit": "GB/s"}}))
+    assert bench.measured_peaks(str(f)) == (6500.0, "measured")
+    f.write_text(json.dumps({"bf16_tflops": 1590}))
+    assert bench.measured_peaks(str(f)) == (bench.FALLBACK_HBM_GBS, "fallback")
+    assert bench.measured_peaks(str(tmp_path / "absent.json")) == (bench.FALLBACK_HBM_GBS, "fallback")
