@@ -38,6 +38,7 @@ class MhcError(RuntimeError):
 
 
 def library_path() -> str:
+    """Path of the in-tree CUDA library (``libmhc_b200.so``) this binding loads."""
     return _build.LIB_PATH
 
 
@@ -87,6 +88,7 @@ def lib() -> ctypes.CDLL:
 
 
 def status_string(status: int) -> str:
+    """Human-readable name of an ``MHC_*`` status code (mhc_status_string)."""
     return lib().mhc_status_string(int(status)).decode()
 
 
