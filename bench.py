@@ -85,7 +85,7 @@ def parse():
     ap.add_argument("--profile", default=None,
                     choices=["newton_fwd", "sinkhorn_fwd", "sinkhorn_bwd", "implicit_bwd", "mix_fwd", "mix_bwd",
                              "proj_mix_fwd", "proj_mix_bwd", "premap_fwd", "mix_post_bwd", "mix_premap_bwd",
-                             "newton_fwd_n", "implicit_bwd_n", "composite_gain"],
+                             "newton_fwd_n", "implicit_bwd_n", "composite_gain", "fwd_bwd_mapped"],
                     help="run one kernel --reps times on one case (for ncu) and exit")
     ap.add_argument("--method", default="newton", help="--profile newton_fwd: projection method")
     ap.add_argument("--layout", default="auto", choices=["auto", "thread", "lane_pair", "row_group"],
@@ -941,6 +941,20 @@ def run_profile_case(args):
         P = api.birkhoff_fwd(A, "newton").reshape(L, args.size, 4, 4)
         fn = lambda: api.composite_gain(P, need_M=False)
         desc = {"layers": L, "tokens": args.size}
+    elif k == "fwd_bwd_mapped":
+        # the zero-copy host path: both kernels read and write pinned host buffers
+        n = args.size
+        if args.dist == "halves_1_10" and n == N_MATS:
+            A_np, G_np = inputs.birkhoff_workload(WORKLOAD)
+        else:
+            A_np, G_np = inputs.birkhoff_logits(n, args.dist, 5), inputs.upstream_grad(n, 6)
+        A_h = torch.from_numpy(A_np).pin_memory()
+        G_h = torch.from_numpy(G_np).pin_memory()
+        P_h = torch.empty_like(A_h).pin_memory()
+        D_h = torch.empty_like(A_h).pin_memory()
+        P_d = torch.empty(A_h.shape, device=dev)
+        fn = lambda: api.birkhoff_fwd_bwd_mapped(A_h, G_h, P_h, D_h, P_d)
+        desc = {"n_mats": n, "dist": args.dist, "path": "mhc_birkhoff_fwd_bwd_mapped"}
     elif k in ("newton_fwd_n", "implicit_bwd_n"):
         cnt = args.size
         A = torch.from_numpy(inputs.birkhoff_logits_n(cnt, args.n, 1.0, 20 + args.n)).to(dev)
