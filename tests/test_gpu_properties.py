@@ -57,3 +57,23 @@ def test_mix_random_shapes(orc, T, cv, seed):
     assert (np.abs(to_np64(out["dh_post"]) - dh).max(1) <= 1e-4 * np.abs(dh).max(1) + 1e-6).all()
     rel, _ = per_matrix_rel_err(to_np64(out["dlogits"]), orc.implicit_bwd(row_normalised(H_np), dH))
     assert rel.max() <= GRAD_REL_TOL, rel.max()
+
+
+@SETTINGS
+@given(n=st.sampled_from([2, 3, 5, 6, 7, 8]), count=st.integers(1, 700), scale=st.sampled_from([0.3, 1.0, 3.0]),
+       seed=st.integers(0, 2 ** 31 - 1), sk_iters=st.integers(1, 30))
+def test_projection_n_random_batches(orc, n, count, scale, seed, sk_iters):
+    # general n: ragged batches (partial tiles of the staged kernels included)
+    rng = np.random.default_rng(seed)
+    A = (rng.standard_normal((count, n, n)) * scale).astype(np.float32)
+    G = rng.standard_normal((count, n, n)).astype(np.float32)
+    P_g = api.birkhoff_fwd_n(to_gpu(A), "newton")
+    P = to_np64(P_g)
+    assert np.abs(P.sum(-1) - 1).max() <= SUM_TOL and np.abs(P.sum(-2) - 1).max() <= SUM_TOL
+    assert np.abs(P - orc.newton(A.astype(np.float64), tol=1e-12, max_iter=200)).max() <= P_ABS_TOL
+    S = to_np64(api.birkhoff_fwd_n(to_gpu(A), "sinkhorn", sk_iters))
+    assert np.abs(S - orc.sinkhorn(A.astype(np.float64), sk_iters)).max() <= P_ABS_TOL
+    dl = to_np64(api.birkhoff_bwd_n(to_gpu(G), P_g))
+    ref = orc.implicit_bwd(row_normalised(P), G.astype(np.float64))
+    rel, _ = per_matrix_rel_err(dl.reshape(count, -1), ref.reshape(count, -1))
+    assert rel.max() <= GRAD_REL_TOL, (n, rel.max())
